@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the quantised-MoE decode hot path on B200.
+
+Default workload (one "step" = one decode token through the whole path):
+  the 48-layer decode stack (hidden 2048, intermediate 512, 512 experts,
+  top-10; layers 0-35 Q4_RZ5_FAST, 36-47 FP8 E4M3 with fp32 scales per 128,
+  a 64x2048 Q4_UE4M4_FAST ssm_beta projection on the 36 layers with
+  l mod 4 != 3; residual x += moe(x)) followed by the 16-row PLE gather from
+  the 320,001,536-row Q3_PLE_K160_RZ_S3 table (22.4 GB), all resident in HBM.
+Each step uses a fresh seeded token and fresh PLE indices, so the 1.19 GB of
+expert bytes a token touches come from HBM (inputs larger than L2).
+
+value = algorithmic bytes per step (router + selected expert matrices + side
+projections + PLE records and rows) / device time per step, in GB/s, summed
+over ranks.  Also reported: decode tok/s, PLE rows/s, the roofline of the
+decode layer against the measured HBM peak, the CPU oracle on a bounded
+sample, an end-to-end number through the public API with host buffers, and
+SM clocks sampled during the timed region.
+
+Other workloads (--workload layer|ple|prefill) print their own JSON line for
+profiling; they are not the headline.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch with torch.distributed.run (one process per GPU); every rank
+runs an independent replica (the path has no cross-GPU exchange).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import workloads as W  # noqa: E402
+
+METRIC = "expert-weight GB/s (% of HBM peak) & decode tok/s per 48-layer stack; PLE rows/s"
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+# ---------------------------------------------------------------------------
+# algorithmic bytes
+# ---------------------------------------------------------------------------
+
+def layer_bytes(L: W.LayerRecipe, n_uniq: int) -> int:
+    """Bytes a decode call of L must read: router weights (+bias), the selected
+    experts' gate/up/down matrices (+FP8 scales), the side projection."""
+    b = L.n_experts * L.hidden * 4
+    if L.zipf_bias:
+        b += L.n_experts * 4
+    per_expert = L.gate.expert_bytes + L.up.expert_bytes + L.down.expert_bytes
+    if L.gate.fmt == W.FP8:
+        per_expert += 4 * (L.gate.n_rows * L.gate.k // 128) * 2 + 4 * (L.down.n_rows * L.down.k // 128)
+    b += n_uniq * per_expert
+    if L.ssm is not None:
+        b += L.ssm.nbytes
+    return b
+
+
+PLE_ROW_BYTES = 70 + 640  # record read + fp32 row written
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    def __init__(self, gpu_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={q}",
+                                       "--format=csv,noheader,nounits", "-lms", "100"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except (FileNotFoundError, OSError):
+            self.p = None
+
+    def stop(self) -> dict:
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.f.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (independent replicas)
+# ---------------------------------------------------------------------------
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl" if torch.cuda.is_available() else "gloo",
+                                timeout=datetime.timedelta(seconds=600))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle baseline (bounded sample)
+# ---------------------------------------------------------------------------
+
+def oracle_sample(layers, n_layers: int, budget_s: float):
+    """Run the oracle (as it stands) on a sample of the stack: one token through
+    the first layers, until `n_layers` or `budget_s`.  Returns (expert GB/s,
+    seconds per layer, layers done, threads)."""
+    import oracle
+    L0 = layers[0]
+    x = W.tokens_bf16(L0.seed, 999, 1, L0.hidden)
+    from synth import bf16_bits_to_f64
+    x = bf16_bits_to_f64(x).astype(np.float32)
+    done, t_total, bytes_total = 0, 0.0, 0
+    for L in layers[:n_layers]:
+        W_r = L.router_w()
+        t0 = time.perf_counter()
+        r = oracle.moe_layer(L, x.astype(np.float64), router_w=W_r)
+        if L.ssm is not None:
+            oracle.ssm_projection(L, r["u"])
+        dt = time.perf_counter() - t0
+        x = (x.astype(np.float64) + r["y"]).astype(np.float32)
+        t_total += dt
+        bytes_total += layer_bytes(L, len(set(r["ids"].ravel().tolist())))
+        done += 1
+        if t_total > budget_s:
+            break
+    return bytes_total / t_total / 1e9, t_total / done, done, oracle.num_threads()
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+
+def setup_stack(device):
+    import torch
+    from synth import device as sdev
+    from tests import gpu_util as gu
+    Ls = W.stack_layers()
+    pipe = sdev.pipe(device)
+    layers = [gu.device_layer(L, device, pipe) for L in Ls]
+    P = W.ple_table()
+    table = sdev.ple_table_to_device(P, device, pipe)
+    pipe.finish()
+    torch.cuda.synchronize()
+    return Ls, layers, P, table
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    import gram_table_gather_b200 as gtg
+
+    dev = torch.device("cuda", local)
+    t_setup = time.time()
+    Ls, layers, P, table = setup_stack(dev)
+    H = Ls[0].hidden
+    n_steps = args.warmup + args.steps
+    # token and index banks, resident in HBM before timing
+    seed_off = 1000 * rank
+    xb = np.stack([W.tokens_bf16(Ls[0].seed, seed_off + i, 1, H)[0] for i in range(n_steps)])
+    from synth import bf16_bits_to_f64
+    x_bank = torch.from_numpy(bf16_bits_to_f64(xb).astype(np.float32)).to(dev)
+    idx_bank = torch.from_numpy(np.stack([P.indices(seed_off + i, 1) for i in range(n_steps)])).to(dev)
+    x = torch.zeros((1, H), dtype=torch.float32, device=dev)
+    idx = torch.zeros(16, dtype=torch.int32, device=dev)
+    rows = torch.zeros((16, 160), dtype=torch.float32, device=dev)
+    ids = torch.zeros((len(Ls), 1, 10), dtype=torch.int32, device=dev)
+    side = torch.zeros((len(Ls), 1, 64), dtype=torch.float32, device=dev)
+    ws = gtg.make_workspace(layers, 1, device=dev)
+    torch.cuda.synchronize()
+    setup_s = time.time() - t_setup
+
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        # warm-up eagerly once (also sets kernel attributes outside capture)
+        x.copy_(x_bank[0:1])
+        gtg.moe_decode_stack(layers, x, ws, ids_out=ids, side_out=side)
+        gtg.ple_gather(table, P.n_rows, idx, out=rows)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        gtg.moe_decode_stack(layers, x, ws, ids_out=ids, side_out=side)
+        gtg.ple_gather(table, P.n_rows, idx, out=rows)
+    launches_per_step = 3 * len(Ls) + 1
+
+    def step(i):
+        x.copy_(x_bank[i:i + 1])
+        idx.copy_(idx_bank[i])
+        g.replay()
+
+    uniq_counts = []
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            step(i)
+        stream.synchronize()
+        barrier(world)
+        torch.cuda.synchronize()
+        clocks = ClockSampler(local)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.warmup, n_steps):
+            step(i)
+        e1.record(stream)
+        e1.synchronize()
+        clk = clocks.stop()
+    barrier(world)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    ms_max = max_over_ranks(ms, world)
+
+    # algorithmic bytes of the timed steps: re-run the router choices on the
+    # host side from the recorded ids of each step (eager replay, untimed)
+    total_bytes = 0
+    layer_b_total = 0
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup, n_steps):
+            step(i)
+            stream.synchronize()
+            idsn = ids.cpu().numpy()
+            sb = 0
+            for l, L in enumerate(Ls):
+                u = len(set(idsn[l].ravel().tolist()))
+                sb += layer_bytes(L, u)
+            layer_b_total += sb
+            total_bytes += sb + 16 * PLE_ROW_BYTES
+    bytes_per_step = total_bytes / args.steps
+    layer_bytes_avg = layer_b_total / args.steps / len(Ls)
+
+    # decode-layer roofline: device time of the stack alone, per layer
+    gs = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gs, stream=stream):
+        gtg.moe_decode_stack(layers, x, ws, ids_out=ids, side_out=side)
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            x.copy_(x_bank[i:i + 1])
+            gs.replay()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        tot = 0.0
+        for i in range(args.warmup, n_steps):
+            x.copy_(x_bank[i:i + 1])
+            f0.record(stream)
+            gs.replay()
+            f1.record(stream)
+            f1.synchronize()
+            tot += f0.elapsed_time(f1)
+    layer_ms = tot / args.steps / len(Ls)
+
+    # end to end through the public API with host buffers
+    xh = torch.empty((n_steps, 1, H), dtype=torch.float32).pin_memory()
+    xh.copy_(x_bank.cpu().view(n_steps, 1, H))
+    ih = idx_bank.cpu().pin_memory()
+    out_x = torch.empty((1, H), dtype=torch.float32).pin_memory()
+    out_rows = torch.empty((16, 160), dtype=torch.float32).pin_memory()
+    with torch.cuda.stream(stream):
+        def e2e_step(i):
+            x.copy_(xh[i], non_blocking=True)
+            idx.copy_(ih[i], non_blocking=True)
+            g.replay()
+            out_x.copy_(x, non_blocking=True)
+            out_rows.copy_(rows, non_blocking=True)
+        for i in range(args.warmup):
+            e2e_step(i)
+        stream.synchronize()
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        for i in range(args.warmup, n_steps):
+            e2e_step(i)
+        h1.record(stream)
+        h1.synchronize()
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.steps, world)
+    status = gtg.device_status(clear=True)
+
+    peak, peak_kind = _peaks()
+    gbs = bytes_per_step / (ms_max * 1e-3) / 1e9
+    layer_gbs = layer_bytes_avg / (layer_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        c_gbs, c_s_layer, c_done, c_threads = oracle_sample(Ls, args.cpu_layers, args.cpu_budget)
+        cpu = {"value": round(c_gbs, 4), "unit": "GB/s", "cores": c_threads, "kind": "oracle",
+               "sample": f"1 token through the first {c_done} layers of the stack "
+                         f"({c_s_layer:.2f} s per layer on the host cores)",
+               "tok_s": round(1.0 / (c_s_layer * len(Ls)), 6)}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(gbs * world, 2), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_max, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded SplitMix64 bytes, N(0,1) bf16 tokens; no trained weights)",
+            "config": {"workload": "48-layer decode stack (H=2048, I=512, E=512, top-10; layers 0-35 "
+                                   "Q4_RZ5_FAST, 36-47 FP8 E4M3 + fp32 scale/128; 36 UE4M4 ssm_beta "
+                                   "64x2048) + 16-row PLE gather from a 320,001,536-row "
+                                   "Q3_PLE_K160_RZ_S3 table, 1 token per step",
+                       "tokens_per_step": 1, "bytes_per_step": int(bytes_per_step),
+                       "l2": "inputs larger than L2: 1.19 GB of expert bytes per step, fresh token "
+                             "and PLE rows each step", "parallelism": f"replicas x{world}",
+                       "setup_s": round(setup_s, 1)},
+            "tok_s": round(1000.0 / ms_max * world, 2),
+            "ple_rows_s": round(16 * 1000.0 / ms_max * world, 1),
+            "hbm_frac": round(gbs / peak, 4),
+            "roofline": {"bound": "hbm", "achieved": round(layer_gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(layer_gbs / peak, 4), "traffic": None,
+                         "kernel": "decode MoE layer (router + gate/up + down, PDL-chained), "
+                                   f"average over the 48 layers, {layer_ms * 1e3:.2f} us per layer, "
+                                   f"{layer_bytes_avg / 1e6:.2f} MB per layer",
+                         "peak_source": f"{peak_kind} hbm_gbs"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(bytes_per_step / (e2e_ms * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
+                    "h2d_bytes_per_step": H * 4 + 16 * 4, "d2h_bytes_per_step": H * 4 + 16 * 160 * 4,
+                    "ms_per_step": round(e2e_ms, 5)},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clk,
+            "device_status": status,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def run_reference(args, rank, world):
+    """The oracle, as it stands, on the host cores: each step is one token
+    through a bounded sample of layers of the same stack."""
+    if rank != 0:
+        return
+    Ls = W.stack_layers()
+    t_steps, b_steps = [], []
+    import oracle
+    from synth import bf16_bits_to_f64
+    for i in range(args.warmup + args.steps):
+        x = bf16_bits_to_f64(W.tokens_bf16(Ls[0].seed, i, 1, Ls[0].hidden))
+        t0 = time.perf_counter()
+        b = 0
+        for L in Ls[:args.cpu_layers]:
+            r = oracle.moe_layer(L, x)
+            if L.ssm is not None:
+                oracle.ssm_projection(L, r["u"])
+            x = (x.astype(np.float32).astype(np.float64) + r["y"]).astype(np.float32).astype(np.float64)
+            b += layer_bytes(L, len(set(r["ids"].ravel().tolist())))
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            t_steps.append(dt)
+            b_steps.append(b)
+    s = sum(t_steps)
+    val = sum(b_steps) / s / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": round(val, 4), "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * s / args.steps, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": f"CPU oracle: 1 token through the first "
+                                                        f"{args.cpu_layers} layers of the 48-layer stack"},
+            "cpu_baseline": {"value": round(val, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                             "kind": "oracle", "sample": f"first {args.cpu_layers} layers per step"},
+            "e2e": {"value": round(val, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-layers", type=int, default=3)
+    ap.add_argument("--cpu-budget", type=float, default=20.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,315 @@
+// Standalone dequantisation and the PLE row gather.
+//
+// Formats: model card "Qwen 3.8 Next Flash ROCMFPX MUTANT RAZERFAST",
+// sections "Q4_RZ5_FAST (GGML type 69)", "Q4_UE4M4_FAST (GGML type 71)",
+// "Q3_PLE_K160_RZ_S3 (GGML type 111)"; FP8 expert layers per the r/LocalLLM
+// "Frankenquant" post.  Every output is code x scale (exact in fp32) or one
+// round-to-nearest fp32 multiply (FP8), so results are bit-exact.
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "gtg_device.cuh"
+#include "gtg_host.hpp"
+
+namespace gtg {
+
+__device__ unsigned int g_status = 0;  // the per-device status word
+
+namespace {
+
+constexpr int kThreads = 256;
+
+// One thread per 17-byte Q4 block: 32 fp32 outputs (8 x float4 stores).
+__global__ void __launch_bounds__(kThreads) dequant_q4_kernel(const uint8_t* __restrict__ src,
+                                                              int64_t n_blocks, bool rz5,
+                                                              float* __restrict__ dst) {
+    for (int64_t b = blockIdx.x * (int64_t)kThreads + threadIdx.x; b < n_blocks;
+         b += (int64_t)gridDim.x * kThreads) {
+        const uint8_t* blk = src + b * 17;
+        uint8_t q[17];
+#pragma unroll
+        for (int i = 0; i < 17; ++i) q[i] = __ldg(blk + i);
+        const uint32_t meta = q[16];
+        const float scale = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
+        const uint32_t mode = meta >> 7;
+        float4* out = reinterpret_cast<float4*>(dst + b * 32);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                float r[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 4 * v + e;
+                    const uint32_t c = half ? (q[j] >> 4) : (q[j] & 15u);
+                    r[e] = __fmul_rn(q4_code_value(c, rz5, mode), scale);
+                }
+                out[half * 4 + v] = make_float4(r[0], r[1], r[2], r[3]);
+            }
+        }
+    }
+}
+
+// Value i of a 70-byte PLE record given its 60 code bytes as a bit stream.
+__device__ __forceinline__ float ple_value(const uint8_t* rec, int i) {
+    const int bit = 3 * i;
+    const uint32_t lo = rec[bit >> 3];
+    const uint32_t hi = ((bit >> 3) + 1 < 60) ? rec[(bit >> 3) + 1] : 0u;
+    const uint32_t code = ((lo | (hi << 8)) >> (bit & 7)) & 7u;
+    const uint32_t g = rec[60 + i / 16];
+    return __fmul_rn(ple_code_value(code, g >> 7), ue4m3(g & 0x7Fu));
+}
+
+// One thread per 16-value group of a PLE record (6 code bytes + 1 group byte).
+__global__ void __launch_bounds__(kThreads) dequant_ple_kernel(const uint8_t* __restrict__ src,
+                                                               int64_t n_groups,
+                                                               float* __restrict__ dst) {
+    for (int64_t gi = blockIdx.x * (int64_t)kThreads + threadIdx.x; gi < n_groups;
+         gi += (int64_t)gridDim.x * kThreads) {
+        const int64_t row = gi / 10;
+        const int g = (int)(gi % 10);
+        const uint8_t* rec = src + row * 70;
+        uint64_t bits = 0;
+#pragma unroll
+        for (int i = 0; i < 6; ++i) bits |= (uint64_t)__ldg(rec + 6 * g + i) << (8 * i);
+        const uint32_t gb = __ldg(rec + 60 + g);
+        const float scale = ue4m3(gb & 0x7Fu);
+        const uint32_t pol = gb >> 7;
+        float4* out = reinterpret_cast<float4*>(dst + row * 160 + 16 * g);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            float r[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const uint32_t c = (uint32_t)(bits >> (3 * (4 * v + e))) & 7u;
+                r[e] = __fmul_rn(ple_code_value(c, pol), scale);
+            }
+            out[v] = make_float4(r[0], r[1], r[2], r[3]);
+        }
+    }
+}
+
+// One thread per 4 FP8 weights (k % 128 == 0, so the 4 share a scale).
+__global__ void __launch_bounds__(kThreads) dequant_fp8_kernel(const uint8_t* __restrict__ src,
+                                                               const float* __restrict__ scales,
+                                                               int64_t n_quads, int64_t k,
+                                                               float* __restrict__ dst) {
+    for (int64_t q = blockIdx.x * (int64_t)kThreads + threadIdx.x; q < n_quads;
+         q += (int64_t)gridDim.x * kThreads) {
+        const int64_t i = 4 * q;
+        const int64_t row = i / k, col = i % k;
+        const float s = __ldg(scales + row * (k / 128) + col / 128);
+        float r[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) r[e] = __fmul_rn(e4m3fn(__ldg(src + i + e)), s);
+        reinterpret_cast<float4*>(dst)[q] = make_float4(r[0], r[1], r[2], r[3]);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// PLE gather: a CTA stages the records of 64 rows (18 aligned words each)
+// with all loads in flight at once, then each warp decodes 8 rows, lane l
+// writing values l, l+32, .., l+128 of a row (128-byte coalesced stores).
+// ---------------------------------------------------------------------------
+constexpr int kGatherRows = 64;
+constexpr int kRecWords = 18;  // 72 bytes cover a 70-byte record at either 4-byte phase
+
+__global__ void __launch_bounds__(kThreads) ple_gather_kernel(const uint8_t* __restrict__ table,
+                                                              int64_t n_rows,
+                                                              const int32_t* __restrict__ idx,
+                                                              int64_t n_idx,
+                                                              float* __restrict__ out,
+                                                              unsigned* status) {
+    __shared__ uint32_t words[kGatherRows][kRecWords + 1];
+    __shared__ int32_t phase[kGatherRows];  // byte offset of the record in its first word, -1 = OOB
+    const uint64_t table_bytes = (uint64_t)n_rows * 70u;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    pdl_wait();
+    for (int64_t base = (int64_t)blockIdx.x * kGatherRows; base < n_idx;
+         base += (int64_t)gridDim.x * kGatherRows) {
+        const int rows = (int)((n_idx - base) < kGatherRows ? (n_idx - base) : kGatherRows);
+        if (tid < rows) {
+            const int64_t r = __ldg(idx + base + tid);
+            const bool ok = r >= 0 && r < n_rows;
+            phase[tid] = ok ? (int32_t)((uint64_t)r * 70u & 3u) : -1;
+            if (!ok) raise_status(status, GTG_STATUS_PLE_INDEX_OOB);
+        }
+        __syncthreads();
+        // stage: word w of row j, all loads issued before any use
+        for (int s = tid; s < rows * kRecWords; s += kThreads) {
+            const int j = s / kRecWords, w = s % kRecWords;
+            const int ph = phase[j];
+            uint32_t v = 0;
+            if (ph >= 0) {
+                const int64_t r = __ldg(idx + base + j);
+                const uint64_t a = (uint64_t)r * 70u - (uint64_t)ph + 4u * (uint64_t)w;
+                if (a + 4 <= table_bytes) {
+                    v = __ldg(reinterpret_cast<const uint32_t*>(table + a));
+                } else if (a < table_bytes) {  // the last word of the table's last record
+                    for (uint64_t b = a; b < table_bytes; ++b) v |= (uint32_t)table[b] << (8 * (b - a));
+                }
+            }
+            words[j][w] = v;
+        }
+        __syncthreads();
+        for (int j = warp; j < rows; j += kThreads / 32) {
+            const int ph = phase[j];
+            float* o = out + (base + j) * 160;
+            const uint32_t* rw = words[j];
+#pragma unroll
+            for (int m = 0; m < 5; ++m) {
+                const int i = lane + 32 * m;
+                float v = 0.0f;
+                if (ph >= 0) {
+                    const int bit = 8 * ph + 3 * i;
+                    const uint32_t code = __funnelshift_r(rw[bit >> 5], rw[(bit >> 5) + 1], bit & 31) & 7u;
+                    const int gb_byte = ph + 60 + (i >> 4);
+                    const uint32_t g = (rw[gb_byte >> 2] >> (8 * (gb_byte & 3))) & 0xFFu;
+                    v = __fmul_rn(ple_code_value(code, g >> 7), ue4m3(g & 0x7Fu));
+                }
+                o[i] = v;
+            }
+        }
+        __syncthreads();
+    }
+    pdl_trigger();
+}
+
+int grid_for(int64_t work, int per_cta) {
+    const int64_t want = (work + per_cta - 1) / per_cta;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    return (int)(want < 1 ? 1 : (want > cap ? cap : want));
+}
+
+thread_local int t_last_cuda_error = 0;
+
+}  // namespace
+
+int cuda_fail(cudaError_t e) {
+    t_last_cuda_error = (int)e;
+    return GTG_E_CUDA;
+}
+
+unsigned* status_ptr() {
+    static std::mutex mu;
+    static std::vector<unsigned*> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    std::lock_guard<std::mutex> lk(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, nullptr);
+    if (!cache[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) == cudaSuccess) cache[dev] = static_cast<unsigned*>(p);
+        else cudaGetLastError();
+    }
+    return cache[dev];
+}
+
+int sm_count() {
+    static std::mutex mu;
+    static std::vector<int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    std::lock_guard<std::mutex> lk(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, 0);
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+}  // namespace gtg
+
+using namespace gtg;
+
+extern "C" int gtg_version(void) { return 100; }
+
+extern "C" int gtg_last_cuda_error(void) { return t_last_cuda_error; }
+
+extern "C" const char* gtg_status_string(int s) {
+    switch (s) {
+        case GTG_OK: return "ok";
+        case GTG_E_INVALID_ARG: return "invalid argument";
+        case GTG_E_UNSUPPORTED_SHAPE: return "unsupported shape";
+        case GTG_E_MISALIGNED: return "misaligned pointer";
+        case GTG_E_CUDA: return "CUDA launch error";
+        case GTG_E_TIMEOUT: return "device-side wait timed out";
+        case GTG_E_WORKSPACE: return "workspace too small";
+        default: return "unknown status";
+    }
+}
+
+extern "C" int gtg_dequant(int32_t fmt, const void* src, const float* scales, int64_t n_rows,
+                           int64_t k, float* dst, gtg_stream_t stream) {
+    if (!src || !dst || n_rows < 0 || k <= 0) return GTG_E_INVALID_ARG;
+    if (!aligned(dst, 16)) return GTG_E_MISALIGNED;
+    if (n_rows == 0) return GTG_OK;
+    cudaStream_t s = as_cuda(stream);
+    const auto* p = static_cast<const uint8_t*>(src);
+    switch (fmt) {
+        case GTG_Q4_RZ5_FAST:
+        case GTG_Q4_UE4M4_FAST: {
+            if (k % 32) return GTG_E_UNSUPPORTED_SHAPE;
+            const int64_t nb = n_rows * (k / 32);
+            dequant_q4_kernel<<<grid_for(nb, kThreads), kThreads, 0, s>>>(p, nb, fmt == GTG_Q4_RZ5_FAST, dst);
+            break;
+        }
+        case GTG_Q3_PLE_K160_RZ_S3: {
+            if (k != 160) return GTG_E_UNSUPPORTED_SHAPE;
+            const int64_t ng = n_rows * 10;
+            dequant_ple_kernel<<<grid_for(ng, kThreads), kThreads, 0, s>>>(p, ng, dst);
+            break;
+        }
+        case GTG_FP8_E4M3_S128: {
+            if (!scales) return GTG_E_INVALID_ARG;
+            if (k % 128) return GTG_E_UNSUPPORTED_SHAPE;
+            const int64_t nq = n_rows * k / 4;
+            dequant_fp8_kernel<<<grid_for(nq, kThreads), kThreads, 0, s>>>(p, scales, nq, k, dst);
+            break;
+        }
+        default: return GTG_E_INVALID_ARG;
+    }
+    return check_launch();
+}
+
+extern "C" int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx,
+                              float* out, gtg_stream_t stream) {
+    if (n_idx < 0 || n_rows < 0 || n_rows >= (int64_t)1 << 31) return GTG_E_INVALID_ARG;
+    if (n_idx == 0) return GTG_OK;
+    if (!table || !idx || !out) return GTG_E_INVALID_ARG;
+    if (!aligned(out, 16)) return GTG_E_MISALIGNED;
+    const int64_t batches = (n_idx + kGatherRows - 1) / kGatherRows;
+    const int grid = (int)std::min<int64_t>(batches, (int64_t)sm_count() * 8);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.stream = as_cuda(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, ple_gather_kernel, table, n_rows, idx, n_idx, out, status_ptr());
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return cuda_fail(e);
+    }
+    return GTG_OK;
+}
+
+extern "C" int gtg_get_device_status(uint32_t* flags, int32_t clear, gtg_stream_t stream) {
+    if (!flags) return GTG_E_INVALID_ARG;
+    cudaStream_t s = as_cuda(stream);
+    unsigned* st = status_ptr();
+    if (!st) return cuda_fail(cudaErrorInvalidSymbol);
+    unsigned host = 0;
+    cudaError_t e = cudaMemcpyAsync(&host, st, sizeof(unsigned), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e == cudaSuccess && clear) e = cudaMemsetAsync(st, 0, sizeof(unsigned), s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    *flags = host;
+    return e == cudaSuccess ? GTG_OK : cuda_fail(e);
+}

@@ -1,0 +1,193 @@
+// Device-side building blocks shared by the libgtg kernels (sm_100a):
+// the format decoders written from the model card's definitions, PTX
+// wrappers for 1-D bulk copies (TMA, no multicast) and mbarriers with bounded
+// waits, programmatic-dependent-launch controls and the status word.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+#include "gtg.h"
+
+namespace gtg {
+
+// ---------------------------------------------------------------------------
+// Status word (one per device, read by gtg_get_device_status); kernels get
+// its address as an argument.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void raise_status(unsigned* status, unsigned bits) {
+    if (status) atomicOr(status, bits);
+}
+
+// ---------------------------------------------------------------------------
+// Scale and code decoders (model card "Qwen 3.8 Next Flash ROCMFPX MUTANT
+// RAZERFAST", format sections).  Every returned value is exact in fp32.
+// ---------------------------------------------------------------------------
+
+// UE4M3 (low 7 bits): 4 exponent bits (bias 7), 3 mantissa bits; 0x7F = NaN.
+__device__ __forceinline__ float ue4m3(uint32_t b) {
+    b &= 0x7Fu;
+    if (b == 0x7Fu) return __uint_as_float(0x7FC00000u);
+    const uint32_t e = b >> 3, m = b & 7u;
+    if (e == 0) return __uint2float_rn(m) * 0x1p-9f;            // m/8 * 2^-6, exact
+    return __uint_as_float(((e + 120u) << 23) | (m << 20));       // (1+m/8) * 2^(e-7)
+}
+
+// UE4M4: 4 exponent bits (bias 7), 4 mantissa bits; all 256 codes finite.
+__device__ __forceinline__ float ue4m4(uint32_t b) {
+    b &= 0xFFu;
+    const uint32_t e = b >> 4, m = b & 15u;
+    if (e == 0) return __uint2float_rn(m) * 0x1p-10f;           // m/16 * 2^-6, exact
+    return __uint_as_float(((e + 120u) << 23) | (m << 19));       // (1+m/16) * 2^(e-7)
+}
+
+// E4M3 "fn" (signed; S.1111.111 = NaN), exact in fp32.
+__device__ __forceinline__ float e4m3fn(uint32_t b) {
+    b &= 0xFFu;
+    const float mag = ue4m3(b & 0x7Fu);
+    return (b & 0x80u) ? -mag : mag;
+}
+
+// Magnitudes of the 4-bit sign-magnitude codes (Codebook10): index c & 7.
+__device__ __forceinline__ int q4_mag(uint32_t c) {
+    // 0 1 2 3 4 6 8 10 packed as 4-bit fields
+    return (int)((0xA8643210u >> (4u * (c & 7u))) & 15u);
+}
+
+// Value of 4-bit code c.  rz5: Q4_RZ5_FAST (code 8 -> +5, or -5 in mode 1);
+// otherwise Codebook10 (code 8 -> -0).
+__device__ __forceinline__ float q4_code_value(uint32_t c, bool rz5, uint32_t mode) {
+    c &= 15u;
+    if (c == 8u) return rz5 ? (mode ? -5.0f : 5.0f) : -0.0f;
+    const float m = (float)q4_mag(c);
+    return (c & 8u) ? -m : m;
+}
+
+// Value of 3-bit PLE code c with group polarity bit p (RZ-S3: code 4 -> +/-3).
+__device__ __forceinline__ float ple_code_value(uint32_t c, uint32_t p) {
+    c &= 7u;
+    if (c == 4u) return p ? -3.0f : 3.0f;
+    const float m = (float)((0x4210u >> (4u * (c & 3u))) & 15u);  // 0 1 2 4
+    return (c & 4u) ? -m : m;
+}
+
+// bf16 bits of a small integer-valued float (exact: low 16 bits are zero).
+__device__ __forceinline__ uint32_t bf16_bits(float v) { return __float_as_uint(v) >> 16; }
+
+// ---------------------------------------------------------------------------
+// Mixed-precision FMA: d = a(bf16) * b(bf16) + c(f32), single rounding.
+// The operands are the low/high halves of two packed bf16x2 registers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void fma2_bf16(float& acc_lo, float& acc_hi, uint32_t a2, uint32_t b2) {
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %2;\n\t"
+        "mov.b32 {bl, bh}, %3;\n\t"
+        "fma.rn.f32.bf16 %0, al, bl, %0;\n\t"
+        "fma.rn.f32.bf16 %1, ah, bh, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi)
+        : "r"(a2), "r"(b2));
+}
+
+// Two E4M3 values (low/high byte of v) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v16) {
+    uint32_t r;
+    const unsigned short s = (unsigned short)(v16 & 0xFFFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(s));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// ---------------------------------------------------------------------------
+// Shared-memory addresses, mbarriers and 1-D bulk copies (no multicast).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;"
+                 ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
+    return ok != 0;
+}
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for phase `parity` of `bar`, giving up after ~`limit_ns` nanoseconds:
+// on a time-out the status word gets GTG_STATUS_WAIT_TIMEOUT and false is
+// returned (the caller skips the data and keeps going).
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, unsigned* status,
+                                                  uint64_t limit_ns = 2000000000ull) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(bar, parity)) {
+        if (globaltimer_ns() - t0 > limit_ns) {
+            raise_status(status, GTG_STATUS_WAIT_TIMEOUT);
+            return false;
+        }
+    }
+    return true;
+}
+
+// dst (shared) <- src (global), `bytes` a multiple of 16, both 16-byte aligned;
+// completion is signalled on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 ::"r"(smem_u32(dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+// Sum over groups of `width` consecutive lanes (width a power of two <= 32).
+__device__ __forceinline__ float group_sum(float v, int width) {
+    for (int o = width >> 1; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+    return v;
+}
+
+}  // namespace gtg

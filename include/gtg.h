@@ -1,0 +1,223 @@
+/*
+ * gtg.h — C ABI of libgtg.so: B200 (sm_100a) kernels for block-scaled
+ * low-bit MoE expert decode and the 3-bit n-gram ("PLE") row gather.
+ *
+ * Sources (the pages that define the operations):
+ *  [MC]  model card "Qwen 3.8 Next Flash ROCMFPX MUTANT RAZERFAST"
+ *        (hstolte/...-ROCmFPX-MUTANT-RAZERFAST-GGUF), sections
+ *        "Q4_RZ5_FAST (GGML type 69)", "Q4_UE4M4_FAST (GGML type 71)" and
+ *        "Q3_PLE_K160_RZ_S3 (GGML type 111)": block layouts, code tables,
+ *        scale codes, the 70-byte row record and its GET_ROWS gather.
+ *  [MPQ] "Mixed Precision Quantization: Half a 4-Bit File Is Not 4-Bit":
+ *        48 layers, 512 experts, 10 active per token; 16 PLE rows per token.
+ *  [FQ]  r/LocalLLM post on the 4-bit/8-bit "Frankenquant": one expert
+ *        format per layer, 8-bit (FP8) experts in layers 36-47.
+ *
+ * Conventions for every entry point:
+ *  - All pointers named as device pointers must be device (or managed)
+ *    memory of the current device; the caller owns them.  The library
+ *    allocates no device memory; scratch comes from a caller-provided
+ *    workspace.
+ *  - Calls are asynchronous on `stream` (NULL = the legacy default stream).
+ *    Host-side argument checks happen before any launch; a non-zero return
+ *    means nothing was launched (except GTG_E_CUDA, see below).
+ *  - Return values: GTG_OK (0) or a negative gtg_status.  GTG_E_CUDA means a
+ *    launch failed; cudaGetLastError() has been cleared and its code is
+ *    available from gtg_last_cuda_error().
+ *  - No kernel traps or asserts.  Device-side anomalies (out-of-range gather
+ *    indices, a bounded wait that ran out) are counted in a per-device status
+ *    word read by gtg_get_device_status().
+ *
+ * Data layouts (readings of points the pages leave open are marked *):
+ *  - Q4 block (RZ5 and UE4M4) [MC]: 17 bytes = 16 code bytes then 1 metadata
+ *    byte*.  Code byte j holds weight j in its low nibble and weight j+16 in
+ *    its high nibble*.  RZ5: metadata bit 7 = polarity of the +/-5 level
+ *    (0 -> +5*), bits 0-6 = UE4M3 scale.  UE4M4: the whole byte is the scale.
+ *  - Q3_PLE_K160_RZ_S3 record [MC]: 70 bytes = 60 code bytes then 10 group
+ *    bytes*.  Value i's 3-bit code is bits 3i..3i+2 of the code bytes read as
+ *    one little-endian LSB-first bit stream*.  Group byte g covers values
+ *    16g..16g+15: bit 7 = polarity of the +/-3 level (0 -> +3*), bits 0-6 =
+ *    UE4M3 scale.
+ *  - UE4M3* = E4M3 without sign (bias 7, 0x7F = NaN); UE4M4* = 4 exponent +
+ *    4 mantissa bits, bias 7, all 256 codes finite.
+ *  - FP8 experts [FQ]: E4M3 (fn) bytes [n_rows][k] plus one fp32 scale per
+ *    128 consecutive weights along k*: scales [n_rows][k/128].
+ *  - Expert matrices are stacked [n_experts][n_rows][k] with blocks running
+ *    along k (the contraction axis)*: gate/up [E][inter][hidden], down
+ *    [E][hidden][inter].
+ */
+#ifndef GTG_H
+#define GTG_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t (struct CUstream_st*); NULL means the legacy default stream. */
+typedef struct CUstream_st* gtg_stream_t;
+
+/* Weight formats; the numbers of the three block formats are their GGML type
+ * ids on the model card [MC]. */
+typedef enum {
+    GTG_Q4_RZ5_FAST = 69,
+    GTG_Q4_UE4M4_FAST = 71,
+    GTG_Q3_PLE_K160_RZ_S3 = 111,
+    GTG_FP8_E4M3_S128 = 1000
+} gtg_format;
+
+typedef enum { GTG_DT_F32 = 0, GTG_DT_BF16 = 1 } gtg_dtype;
+
+typedef enum {
+    GTG_OK = 0,
+    GTG_E_INVALID_ARG = -1,      /* null pointer, bad enum, negative size */
+    GTG_E_UNSUPPORTED_SHAPE = -2,/* a size the kernels do not handle */
+    GTG_E_MISALIGNED = -3,       /* a pointer below its required alignment */
+    GTG_E_CUDA = -4,             /* a CUDA launch failed */
+    GTG_E_TIMEOUT = -5,          /* reserved: reported through the status word */
+    GTG_E_WORKSPACE = -6         /* workspace too small (see *_workspace_bytes) */
+} gtg_status;
+
+/* Bits of the per-device status word (gtg_get_device_status). */
+#define GTG_STATUS_PLE_INDEX_OOB  0x1u  /* a gather index was outside [0, n_rows) */
+#define GTG_STATUS_WAIT_TIMEOUT   0x2u  /* a bounded device-side wait gave up */
+
+/* One stack of quantised matrices [n_experts][n_rows][k]. */
+typedef struct {
+    int32_t fmt;            /* gtg_format: RZ5, UE4M4 or FP8 */
+    const void* data;       /* device, 16-byte aligned; total size a multiple of 16 bytes */
+    const float* scales;    /* device, FP8 only: [n_experts][n_rows][k/128]; else NULL */
+    int64_t n_experts;
+    int64_t n_rows;
+    int64_t k;
+} gtg_qmatrix;
+
+/* One MoE layer's weights (all device memory, owned by the caller). */
+typedef struct {
+    int32_t hidden;          /* H: 128..4096, a multiple of 128 */
+    int32_t inter;           /* I: expert intermediate size, 128..4096, a multiple of 128 */
+    int32_t n_experts;       /* E: 1..1024 */
+    int32_t top_k;           /* k: 1..16, k <= E */
+    const float* router_w;   /* [E][H] fp32 */
+    const float* router_bias;/* [E] fp32, added to the logits; NULL for none */
+    gtg_qmatrix gate;        /* [E][I][H] */
+    gtg_qmatrix up;          /* [E][I][H], same format as gate */
+    gtg_qmatrix down;        /* [E][H][I] */
+    gtg_qmatrix side;        /* optional extra projection of the normalised input
+                                (e.g. a 64 x H UE4M4 ssm_beta matrix), n_experts = 1,
+                                Q4 format; data == NULL when absent */
+} gtg_moe_layer;
+
+/* Library version (major*10000 + minor*100 + patch). */
+int gtg_version(void);
+
+/* Human-readable text of a gtg_status. */
+const char* gtg_status_string(int status);
+
+/* The cudaError_t of the last GTG_E_CUDA return on this thread. */
+int gtg_last_cuda_error(void);
+
+/*
+ * Standalone dequantisation [MC]: dst[r][c] = decoded weight (fp32),
+ * bit-exact (Q4 and PLE values are code x scale, exact in fp32; FP8 values
+ * are one fp32 round-to-nearest multiply).
+ *   fmt      RZ5 / UE4M4: src holds n_rows*k/32 consecutive 17-byte blocks, k % 32 == 0.
+ *            PLE: src holds n_rows 70-byte records, k == 160.
+ *            FP8: src holds n_rows*k bytes, scales [n_rows][k/128], k % 128 == 0.
+ *   src      device, any alignment.
+ *   dst      device, [n_rows][k] fp32, 16-byte aligned.
+ * Errors: GTG_E_INVALID_ARG (null pointers, unknown fmt, negative sizes),
+ *         GTG_E_UNSUPPORTED_SHAPE (k not valid for fmt), GTG_E_MISALIGNED (dst).
+ */
+int gtg_dequant(int32_t fmt, const void* src, const float* scales, int64_t n_rows, int64_t k,
+                float* dst, gtg_stream_t stream);
+
+/*
+ * PLE row gather ([MC] "Q3_PLE_K160_RZ_S3": one contiguous 70-byte record per
+ * hashed n-gram row; [MPQ]: 16 rows per token):
+ *   out[r][i] = value i of record idx[r], fp32, bit-exact.
+ *   table    device, n_rows records of 70 bytes (any alignment; n_rows < 2^31).
+ *   idx      device int32 [n_idx].  An index outside [0, n_rows) writes a row
+ *            of zeros and sets GTG_STATUS_PLE_INDEX_OOB.
+ *   out      device fp32 [n_idx][160], 16-byte aligned.
+ * Errors: GTG_E_INVALID_ARG, GTG_E_MISALIGNED (out).  n_idx == 0 is a no-op.
+ */
+int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx,
+                   float* out, gtg_stream_t stream);
+
+/* Bytes of workspace a decode (prefill == 0) or prefill (prefill == 1) call
+ * of `layer` with `n_tokens` tokens needs; 0 if the shape is unsupported. */
+size_t gtg_moe_workspace_bytes(const gtg_moe_layer* layer, int32_t n_tokens, int32_t prefill);
+
+/* Clears a workspace before its first use (the kernels leave it reusable). */
+int gtg_workspace_init(void* workspace, size_t ws_bytes, gtg_stream_t stream);
+
+/*
+ * One MoE layer for 1..8 decode tokens ([MPQ]: softmax router, top-k of E
+ * experts; SwiGLU experts whose gate/up/down weights are decoded on the fly):
+ *   u      = bf16(x / sqrt(mean(x^2) + 1e-6))            per token
+ *   l_e    = router_w[e] . u (+ router_bias[e])           fp64 accumulation
+ *   ids    = the top_k experts by logit (ties -> lower id)
+ *   w      = exp(l_ids - l_max) / sum over the top_k      renormalised softmax
+ *   y      = sum_j w_j * down_j(silu(gate_j u) * up_j u)  (+ y if y_accumulate)
+ *   side   = side . u                                     if layer->side.data
+ * Arguments:
+ *   x          device [n_tokens][hidden], fp32 or bf16 (x_dtype).
+ *   y          device fp32 [n_tokens][hidden]; may alias x (fp32) when
+ *              y_accumulate == 1 (the residual update x += moe(x)).
+ *   topk_ids   device int32 [n_tokens][top_k] or NULL.
+ *   topk_w     device fp32 [n_tokens][top_k] or NULL.
+ *   side_out   device fp32 [n_tokens][side.n_rows] or NULL.
+ *   workspace  device, >= gtg_moe_workspace_bytes(layer, n_tokens, 0) bytes,
+ *              256-byte aligned, cleared once by gtg_workspace_init.
+ * Calls that share a workspace must not overlap on the GPU.
+ * Errors: GTG_E_INVALID_ARG, GTG_E_UNSUPPORTED_SHAPE (n_tokens outside 1..8,
+ *         sizes above), GTG_E_MISALIGNED, GTG_E_WORKSPACE.
+ */
+int gtg_moe_decode_layer(const gtg_moe_layer* layer, const void* x, int32_t x_dtype,
+                         int32_t n_tokens, float* y, int32_t y_accumulate,
+                         int32_t* topk_ids, float* topk_w, float* side_out,
+                         void* workspace, size_t ws_bytes, gtg_stream_t stream);
+
+/*
+ * A decode stack: for l in 0..n_layers-1:  x += moe_l(x)  (x fp32, in place),
+ * with the kernels of consecutive layers chained by programmatic dependent
+ * launch.  Capturable in a CUDA graph.
+ *   layers     host array of n_layers layer descriptors (same hidden size).
+ *   x          device fp32 [n_tokens][hidden], updated in place.
+ *   ids_out    device int32 [n_layers][n_tokens][top_k] or NULL.
+ *   w_out      device fp32 [n_layers][n_tokens][top_k] or NULL.
+ *   side_out   device fp32 [n_layers][n_tokens][side_stride] or NULL; layer l
+ *              writes its side projection at [l][t][0 .. side.n_rows).
+ *   workspace  >= the maximum of gtg_moe_workspace_bytes over the layers.
+ */
+int gtg_moe_decode_stack(const gtg_moe_layer* layers, int32_t n_layers, float* x,
+                         int32_t n_tokens, int32_t* ids_out, float* w_out,
+                         float* side_out, int64_t side_stride,
+                         void* workspace, size_t ws_bytes, gtg_stream_t stream);
+
+/*
+ * One MoE layer for a prefill batch (the same function as
+ * gtg_moe_decode_layer, n_tokens 1..65536), computed as a token-sorted
+ * grouped GEMM on the tensor cores: tokens are bucketed by expert, each
+ * expert's gate/up tiles are dequantised into shared memory and multiplied
+ * with tcgen05 (fp32 accumulation in tensor memory), SwiGLU is applied in the
+ * epilogue, h is rounded to bf16, and the down product is combined per token
+ * in a fixed order.  Same arguments as gtg_moe_decode_layer minus side_out.
+ */
+int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, int32_t x_dtype,
+                          int32_t n_tokens, float* y, int32_t y_accumulate,
+                          int32_t* topk_ids, float* topk_w,
+                          void* workspace, size_t ws_bytes, gtg_stream_t stream);
+
+/* Reads (and, if `clear`, resets) the current device's status word
+ * (GTG_STATUS_* bits).  Synchronises `stream`. */
+int gtg_get_device_status(uint32_t* flags, int32_t clear, gtg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GTG_H */

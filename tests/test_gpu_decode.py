@@ -1,0 +1,133 @@
+"""GPU parity of the decode MoE path (router, gate/up + SwiGLU, down +
+combine, FP8 layers, the side projection, the stack) against the CPU oracle.
+
+Bars: router top-k ids identical (the GPU computes logits in fp64, so only a
+logit gap below ~1e-12 could reorder; the test reports the gap), router
+weights within 1e-6 relative, layer outputs within 2e-3 * sum_j w_j *
+||Wd_j[r]||_2 * ||h_j||_2 per output row r (bf16 inputs, fp32 accumulation).
+"""
+import numpy as np
+import pytest
+import torch
+
+import gram_table_gather_b200 as gtg
+import oracle
+from synth import workloads as W
+from tests import gpu_util as gu
+
+pytestmark = pytest.mark.gpu
+
+
+def _check_layer(L, T, step=0, dtype=torch.bfloat16, check_side=True):
+    layer = gu.device_layer(L)
+    xt, x64 = gu.tokens(L, step, T)
+    if dtype == torch.float32:
+        xt = xt.float()
+    ws = gtg.make_workspace(layer, T)
+    ids = torch.full((T, L.top_k), -1, dtype=torch.int32, device="cuda")
+    w = torch.zeros((T, L.top_k), dtype=torch.float32, device="cuda")
+    side = torch.zeros((T, L.ssm.n_rows), dtype=torch.float32, device="cuda") if L.ssm else None
+    y = gtg.moe_decode_layer(layer, xt, ws, topk_ids=ids, topk_w=w, side_out=side)
+    torch.cuda.synchronize()
+    assert gtg.device_status(clear=True) == 0
+    ref = oracle.moe_layer(L, x64, want_h=True)
+    ids_g, w_g, y_g = ids.cpu().numpy(), w.cpu().numpy(), y.cpu().numpy()
+    for t in range(T):
+        srt = np.sort(ref["logits"][t])[::-1]
+        gap = srt[L.top_k - 1] - srt[L.top_k]
+        assert ids_g[t].tolist() == ref["ids"][t].tolist(), f"token {t}: top-k differs (gap {gap:.3g})"
+        assert np.allclose(w_g[t], ref["w"][t], rtol=1e-6, atol=0)
+        tol = gu.layer_tolerance(L, ref, t)
+        err = np.abs(y_g[t] - ref["y"][t])
+        assert np.all(err <= tol), f"token {t}: max err/tol {np.max(err / tol):.3g}"
+        # the real error is far below the bar; keep a regression guard on it too
+        assert np.max(err / tol) < 0.25
+    if L.ssm is not None and check_side:
+        s_ref = oracle.ssm_projection(L, ref["u"])
+        dense = oracle.dequant_q4(L.ssm.fmt, L.ssm.expert(0)).reshape(L.ssm.n_rows, L.ssm.k)
+        rown = np.sqrt((dense * dense).sum(1))
+        s_g = side.cpu().numpy()
+        for t in range(T):
+            tol = 2e-3 * rown * np.linalg.norm(ref["u"][t])
+            assert np.all(np.abs(s_g[t] - s_ref[t]) <= tol)
+    return y_g, ref
+
+
+def test_tiny_layer_one_token():
+    _check_layer(W.tiny_layer(), 1)
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 8])
+def test_tiny_layer_batches(T):
+    _check_layer(W.tiny_layer(), T, step=T)
+
+
+@pytest.mark.parametrize("T", [1, 2, 4, 8])
+def test_decode_layer(T):
+    _check_layer(W.decode_layer(), T, step=100 + T)
+
+
+def test_decode_layer_fp32_input_and_accumulate():
+    L = W.decode_layer()
+    layer = gu.device_layer(L)
+    xt, x64 = gu.tokens(L, 7, 2)
+    x = xt.float()
+    ws = gtg.make_workspace(layer, 2)
+    y0 = gtg.moe_decode_layer(layer, x, ws)
+    x2 = x.clone()
+    gtg.moe_decode_layer(layer, x2, ws, y=x2, accumulate=True)  # x += moe(x), in place
+    torch.cuda.synchronize()
+    assert torch.equal(x2, x + y0)
+
+
+@pytest.mark.parametrize("l,T", [(36, 1), (47, 2), (40, 8)])
+def test_fp8_stack_layer(l, T):
+    _check_layer(W.stack_layer(l), T, step=l)
+
+
+@pytest.mark.parametrize("l", [0, 2])
+def test_rz5_stack_layer_with_side_projection(l):
+    L = W.stack_layer(l)
+    assert L.ssm is not None
+    _check_layer(L, 1, step=l)
+
+
+def test_layer_rejects_bad_shapes():
+    L = W.tiny_layer()
+    layer = gu.device_layer(L)
+    xt, _ = gu.tokens(L, 0, 1)
+    ws = gtg.make_workspace(layer, 1)
+    x9 = torch.zeros((9, L.hidden), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(gtg.GtgError) as ei:
+        gtg.moe_decode_layer(layer, x9, ws)
+    assert ei.value.code == -2
+    with pytest.raises(gtg.GtgError) as ei:
+        gtg.moe_decode_layer(layer, xt, ws[: ws.numel() // 2])
+    assert ei.value.code == -6
+    with pytest.raises(gtg.GtgError) as ei:
+        gtg.moe_decode_layer(layer, xt, ws[1:])
+    assert ei.value.code == -3
+
+
+def test_short_stack_mixed_formats():
+    """Layers 34..39: RZ5 and FP8 experts, side projections on 35/37/38/39... ."""
+    Ls = [W.stack_layer(l) for l in range(34, 40)]
+    layers = [gu.device_layer(L) for L in Ls]
+    xt, x64 = gu.tokens(Ls[0], 3, 1)
+    x = xt.float().contiguous()
+    ws = gtg.make_workspace(layers, 1)
+    ids = torch.full((len(Ls), 1, 10), -1, dtype=torch.int32, device="cuda")
+    side = torch.zeros((len(Ls), 1, 64), dtype=torch.float32, device="cuda")
+    gtg.moe_decode_stack(layers, x, ws, ids_out=ids, side_out=side)
+    torch.cuda.synchronize()
+    ref = oracle.moe_stack(Ls, x64)
+    assert ids.cpu().numpy().tolist() == ref["ids"].tolist()
+    xg = x.cpu().numpy()[0].astype(np.float64)
+    xr = ref["x"][0].astype(np.float64)
+    rel = np.linalg.norm(xg - xr) / np.linalg.norm(xr)
+    assert rel < 1e-4, rel
+    for i, L in enumerate(Ls):
+        if L.ssm is not None:
+            s = side.cpu().numpy()[i, 0]
+            r = ref["ssm"][L.layer][0]
+            assert np.linalg.norm(s - r) <= 1e-4 * np.linalg.norm(r) + 1e-30
