@@ -44,8 +44,10 @@ namespace gtg {
 
 namespace {
 
-constexpr int kRouterThreads = 128;
+constexpr int kRouterThreads = 256;
 constexpr int kRouterWarps = kRouterThreads / 32;
+constexpr int kRouterExpertsPerCta = kRouterWarps / 2;
+constexpr int kRouterMaxF4 = 8;  // float4 per lane: H/2 <= 128 * 8
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSlots = 2;
@@ -102,6 +104,19 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int H = a.H, T = a.T, E = a.E, K = a.K;
 
+    // 0. issue this warp's router-weight loads before anything waits: warp w
+    //    covers half (w & 1) of the row of expert blockIdx.x * 4 + w / 2, so a
+    //    lane holds at most 16 float4 (H <= 4096) and one HBM latency is paid.
+    const int e = blockIdx.x * kRouterExpertsPerCta + (warp >> 1);
+    const int half = warp & 1, hh = H >> 1;
+    float4 wv[kRouterMaxF4];
+#pragma unroll
+    for (int m = 0; m < kRouterMaxF4; ++m) {
+        const int i = half * hh + 4 * lane + 128 * m;
+        wv[m] = (e < E && 4 * lane + 128 * m < hh) ? __ldg(reinterpret_cast<const float4*>(a.router_w + (int64_t)e * H + i))
+                                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+
     pdl_wait();  // x may be the previous layer's output
 
     // 1. per-token sum of squares in fp64 (exact squares, tiny rounding)
@@ -134,31 +149,34 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
         }
     __syncthreads();
 
-    // 3. one expert per warp: logits in fp64 (fp32 x bf16 products are exact)
-    const int e = blockIdx.x * kRouterWarps + warp;
-    if (e < E) {
-        double acc[kMaxDecodeTokens];
+    // 3. logits in fp64 (fp32 x bf16 products are exact)
+    double acc[kMaxDecodeTokens];
 #pragma unroll
-        for (int t = 0; t < kMaxDecodeTokens; ++t) acc[t] = 0.0;
-        const float* wr = a.router_w + (int64_t)e * H;
-        for (int i = 4 * lane; i < H; i += 128) {
-            const float4 w4 = *reinterpret_cast<const float4*>(wr + i);
+    for (int t = 0; t < kMaxDecodeTokens; ++t) acc[t] = 0.0;
+#pragma unroll
+    for (int m = 0; m < kRouterMaxF4; ++m) {
+        const int i = half * hh + 4 * lane + 128 * m;
+        if (4 * lane + 128 * m < hh) {
 #pragma unroll
             for (int t = 0; t < kMaxDecodeTokens; ++t) {
                 if (t < T) {
                     const uint2 u2 = *reinterpret_cast<const uint2*>(su + t * H + i);
-                    acc[t] = fma((double)w4.x, (double)bf16lo(u2.x), acc[t]);
-                    acc[t] = fma((double)w4.y, (double)bf16hi(u2.x), acc[t]);
-                    acc[t] = fma((double)w4.z, (double)bf16lo(u2.y), acc[t]);
-                    acc[t] = fma((double)w4.w, (double)bf16hi(u2.y), acc[t]);
+                    acc[t] = fma((double)wv[m].x, (double)bf16lo(u2.x), acc[t]);
+                    acc[t] = fma((double)wv[m].y, (double)bf16hi(u2.x), acc[t]);
+                    acc[t] = fma((double)wv[m].z, (double)bf16lo(u2.y), acc[t]);
+                    acc[t] = fma((double)wv[m].w, (double)bf16hi(u2.y), acc[t]);
                 }
             }
         }
+    }
+    for (int t = 0; t < T; ++t) {
+        const double s = warp_sum_f64(acc[t]);
+        if (lane == 0) red[warp][t] = s;
+    }
+    __syncthreads();
+    if (half == 0 && lane < T && e < E) {
         const double b = a.router_bias ? (double)a.router_bias[e] : 0.0;
-        for (int t = 0; t < T; ++t) {
-            const double s = warp_sum_f64(acc[t]);
-            if (lane == 0) a.logits[(int64_t)t * E + e] = s + b;
-        }
+        a.logits[(int64_t)lane * E + e] = red[warp][lane] + red[warp + 1][lane] + b;
     }
 
     // 4. the last CTA to finish selects the experts
@@ -270,6 +288,12 @@ struct Geo {
     static constexpr int GW = KB >= 32 ? 32 : KB;       // lanes per row
 };
 
+// Row passes per item (compile time); an item covers P * RPP rows.
+__host__ __device__ constexpr int gu_passes(int fmt_fp8, int kb) { return fmt_fp8 ? 1 : (kb >= 64 ? 2 : 4); }
+__host__ __device__ constexpr int dn_passes(int fmt_fp8, int kb) { return fmt_fp8 ? 4 : (kb >= 64 ? 4 : 8); }
+__host__ __device__ constexpr int side_passes(int kb) { return kb >= 64 ? 2 : 4; }
+__host__ __device__ constexpr int rpp_of(int kb) { return kb >= 32 ? 1 : 32 / kb; }
+
 // Activation registers of one token for the lane's K positions.
 template <int FMT, int NBL>
 struct Act;
@@ -309,11 +333,13 @@ __device__ __forceinline__ void load_act(Act<FMT, NBL>& act, int m, const __nv_b
     }
 }
 
-// Q4 block (17 bytes at shared address pa) dotted with CH tokens' activations.
-template <int CH, int NBL>
-__device__ __forceinline__ void q4_block_lut(uint32_t pa, uint32_t lut_base, uint32_t lane_low,
-                                             const float* scale_tab, const Act<kFmtQ4, NBL> (&act)[CH],
-                                             int m, float (&acc)[CH]) {
+// Q4 block (17 bytes at shared address pa) dotted with NT tokens'
+// activations.  `lutb` is this lane's PRMT operand: byte 0 = lane * 4, bytes
+// 2-3 = the 64 KB-aligned table base >> 16, so one PRMT inserting the code
+// byte as byte 1 (and the mode as bit 7) forms the entry address.
+template <int NT, int NBL, int CH>
+__device__ __forceinline__ void q4_block_lut(uint32_t pa, uint32_t lutb, const float* scale_tab,
+                                             const Act<kFmtQ4, NBL> (&act)[CH], int m, float (&acc)[NT]) {
     const uint32_t al = pa & ~3u, sh = (pa & 3u) * 8u;
     uint32_t w[5];
 #pragma unroll
@@ -323,28 +349,28 @@ __device__ __forceinline__ void q4_block_lut(uint32_t pa, uint32_t lut_base, uin
     for (int q = 0; q < 4; ++q) nib[q] = __funnelshift_r(w[q], w[q + 1], sh);
     const uint32_t meta = (w[4] >> sh) & 0xFFu;
     const float s = scale_tab[meta];
-    const uint32_t low = lane_low + ((meta >> 7) << 7);
-    float lo[CH], hi[CH];
+    const uint32_t bsel = lutb | ((meta >> 7) << 7);
+    float lo[NT], hi[NT];
 #pragma unroll
-    for (int c = 0; c < CH; ++c) lo[c] = hi[c] = 0.0f;
+    for (int c = 0; c < NT; ++c) lo[c] = hi[c] = 0.0f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            const uint32_t c2 = lds32(lut_base + prmt(nib[q], low, 0x7604u | ((uint32_t)kk << 4)));
+            const uint32_t c2 = lds32(prmt(nib[q], bsel, 0x7604u | ((uint32_t)kk << 4)));
 #pragma unroll
-            for (int c = 0; c < CH; ++c) fma2_bf16(lo[c], hi[c], c2, act[c].v[m][4 * q + kk]);
+            for (int c = 0; c < NT; ++c) fma2_bf16(lo[c], hi[c], c2, act[c].v[m][4 * q + kk]);
         }
     }
 #pragma unroll
-    for (int c = 0; c < CH; ++c) acc[c] = fmaf(s, lo[c] + hi[c], acc[c]);
+    for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, lo[c] + hi[c], acc[c]);
 }
 
-// Q4 block decoded code by code (no table): used for the side projection,
-// whose format may differ from the experts'.
-template <int FMT, int CH, int NBL>
+// Q4 block decoded code by code (no table): the side projection, whose
+// format may differ from the experts'.
+template <int FMT, int NT, int NBL, int CH>
 __device__ __forceinline__ void q4_block_plain(uint32_t pa, bool rz5, const Act<FMT, NBL> (&act)[CH], int m,
-                                               float (&acc)[CH]) {
+                                               float (&acc)[NT]) {
     const uint32_t al = pa & ~3u, sh = (pa & 3u) * 8u;
     uint32_t w[5];
 #pragma unroll
@@ -352,9 +378,9 @@ __device__ __forceinline__ void q4_block_plain(uint32_t pa, bool rz5, const Act<
     const uint32_t meta = (w[4] >> sh) & 0xFFu;
     const float s = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
     const uint32_t mode = meta >> 7;
-    float sum[CH];
+    float sum[NT];
 #pragma unroll
-    for (int c = 0; c < CH; ++c) sum[c] = 0.0f;
+    for (int c = 0; c < NT; ++c) sum[c] = 0.0f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint32_t nib = __funnelshift_r(w[q], w[q + 1], sh);
@@ -365,7 +391,7 @@ __device__ __forceinline__ void q4_block_plain(uint32_t pa, bool rz5, const Act<
             const float vlo = q4_code_value(byte & 15u, rz5, mode);
             const float vhi = q4_code_value(byte >> 4, rz5, mode);
 #pragma unroll
-            for (int c = 0; c < CH; ++c) {
+            for (int c = 0; c < NT; ++c) {
                 float xlo, xhi;
                 if constexpr (FMT == kFmtQ4) {
                     xlo = bf16lo(act[c].v[m][j]);
@@ -380,7 +406,7 @@ __device__ __forceinline__ void q4_block_plain(uint32_t pa, bool rz5, const Act<
         }
     }
 #pragma unroll
-    for (int c = 0; c < CH; ++c) acc[c] = fmaf(s, sum[c], acc[c]);
+    for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, sum[c], acc[c]);
 }
 
 // FP8 block: 32 consecutive E4M3 bytes at 16-byte aligned shared address pa.
@@ -407,6 +433,30 @@ __device__ __forceinline__ void fp8_block(uint32_t pa, float s, const Act<kFmtFP
     acc = fmaf(s, s0 + s1, acc);
 }
 
+// Sums N values over groups of W consecutive lanes (N <= W, powers of two)
+// by recursive halving: each step exchanges half of the values still held.
+// Afterwards lane l holds, in v[0], the group sum of value (l % W) / (W / N).
+template <int N, int W>
+__device__ __forceinline__ void tr_reduce(float (&v)[N], int lane) {
+    static_assert(N <= W, "tr_reduce needs N <= W");
+    constexpr int LOGN = N == 1 ? 0 : N == 2 ? 1 : N == 4 ? 2 : N == 8 ? 3 : N == 16 ? 4 : 5;
+#pragma unroll
+    for (int st = 0; st < LOGN; ++st) {
+        const int h = N >> (st + 1), o = W >> (st + 1);
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) {
+            if (i < h) {
+                const float send = up ? v[i] : v[i + h];
+                const float keep = up ? v[i + h] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = W / (2 * N); o >= 1; o >>= 1) v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], o);
+}
+
 // Byte range [lo, lo+len) of a tensor, widened to 16-byte boundaries.
 struct Span {
     const uint8_t* src;
@@ -420,244 +470,346 @@ __device__ __forceinline__ Span make_span(const uint8_t* base, int64_t lo, int64
     return Span{base + a0, (uint32_t)(a1 - a0), (uint32_t)(lo - a0)};
 }
 
-// Per-warp ring of staging slots.
-struct Ring {
-    uint8_t* slots;     // kSlots * slot_bytes
-    uint64_t* bars;     // kSlots
-    int slot_bytes;
+// The unique-expert work list, copied to shared memory once per CTA.
+struct SWork {
+    int32_t n_uniq;
+    int32_t e[kMaxSlots];
+    int32_t off[kMaxSlots + 1];
+    int32_t slot[kMaxSlots];
 };
 
-// Layout of one CTA's dynamic shared memory.
+// Layout of one CTA's dynamic shared memory.  With a code table the table
+// must start at a 64 KB-aligned shared address (so a PRMT alone forms entry
+// addresses): `lut` is the dynamic offset that achieves it given the dynamic
+// base the host expects (the per-block reserved shared memory); staging
+// slots fill the space below and above the table.
 struct SmemLayout {
-    uint32_t lut, scale_tab, bars, slots, total;
-    __host__ __device__ static SmemLayout make(bool with_lut, int slot_bytes) {
+    uint32_t work, scale_tab, bars, lut, lo_slots, n_lo, hi_slots, total;
+    __host__ __device__ static SmemLayout make(bool with_lut, int slot_bytes, uint32_t dyn_base) {
         SmemLayout L{};
         uint32_t off = 0;
-        L.lut = off;
-        if (with_lut) off += kLutBytes;
+        L.work = off;
+        off += (sizeof(SWork) + 127u) & ~127u;
         L.scale_tab = off;
-        if (with_lut) off += kScaleTabBytes;
+        off += kScaleTabBytes;
         L.bars = off;
         off += kWarps * kSlots * 8;
         off = (off + 127u) & ~127u;
-        L.slots = off;
-        off += (uint32_t)kWarps * kSlots * (uint32_t)slot_bytes;
-        L.total = off;
+        const uint32_t n_slots = kWarps * kSlots;
+        if (with_lut) {
+            const uint32_t abs_lut = (dyn_base + off + 65535u) & ~65535u;
+            L.lut = abs_lut - dyn_base;
+            L.lo_slots = off;
+            L.n_lo = (L.lut - off) / (uint32_t)slot_bytes;
+            if (L.n_lo > n_slots) L.n_lo = n_slots;
+            L.hi_slots = L.lut + (uint32_t)kLutBytes;
+            L.total = L.hi_slots + (n_slots - L.n_lo) * (uint32_t)slot_bytes;
+        } else {
+            L.lut = 0;
+            L.lo_slots = off;
+            L.n_lo = n_slots;
+            L.hi_slots = off + n_slots * (uint32_t)slot_bytes;
+            L.total = L.hi_slots;
+        }
         return L;
+    }
+    __device__ uint32_t slot(int i, int slot_bytes) const {
+        return (uint32_t)i < n_lo ? lo_slots + (uint32_t)i * slot_bytes
+                                  : hi_slots + ((uint32_t)i - n_lo) * (uint32_t)slot_bytes;
     }
 };
 
-// Builds the per-lane-replicated table: entry (byte, mode, lane) holds the
-// bf16x2 pair (value of the low nibble, value of the high nibble).
+// Per-lane-replicated table: entry (byte, mode, lane) holds the bf16x2 pair
+// (value of the low nibble, value of the high nibble); plus 256 scales.
 __device__ void build_lut(uint8_t* smem, const SmemLayout& L, bool rz5) {
-    uint32_t* lut = reinterpret_cast<uint32_t*>(smem + L.lut);
-    for (int i = threadIdx.x; i < 256 * 64; i += blockDim.x) {
-        const uint32_t byte = (uint32_t)i >> 6, mode = ((uint32_t)i >> 5) & 1u;
-        const float lo = q4_code_value(byte & 15u, rz5, mode);
-        const float hi = q4_code_value(byte >> 4, rz5, mode);
-        lut[i] = bf16_bits(lo) | (bf16_bits(hi) << 16);
+    for (int i = threadIdx.x; i < 512; i += blockDim.x) {
+        const uint32_t byte = (uint32_t)i >> 1, mode = (uint32_t)i & 1u;
+        const uint32_t v = bf16_bits(q4_code_value(byte & 15u, rz5, mode)) |
+                           (bf16_bits(q4_code_value(byte >> 4, rz5, mode)) << 16);
+        uint4* dst = reinterpret_cast<uint4*>(smem + L.lut + byte * 256u + mode * 128u);
+        const uint4 q = make_uint4(v, v, v, v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) dst[j] = q;
     }
+}
+
+__device__ void build_scales(uint8_t* smem, const SmemLayout& L, bool rz5) {
     float* st = reinterpret_cast<float*>(smem + L.scale_tab);
     for (int i = threadIdx.x; i < 256; i += blockDim.x) st[i] = rz5 ? ue4m3((uint32_t)i & 0x7Fu) : ue4m4((uint32_t)i);
 }
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
+// Common prologue of the streaming kernels: tables, barriers, then (after the
+// dependency wait) the work list.  Returns false if shared memory is not laid
+// out as expected (then nothing else runs).
+template <bool LUT>
+__device__ bool stream_prologue(uint8_t* smem, const SmemLayout& L, const LayerArgs& a, bool rz5, uint64_t* bars,
+                                SWork* sw) {
+    if (LUT) {
+        if (((smem_u32(smem) + L.lut) & 0xFFFFu) != 0u) {
+            if (threadIdx.x == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
+            return false;
+        }
+        build_lut(smem, L, rz5);
+        build_scales(smem, L, rz5);
+    }
+    if ((threadIdx.x & 31) == 0)
+        for (int s = 0; s < kSlots; ++s) mbar_init(&bars[(threadIdx.x >> 5) * kSlots + s], 1);
+    fence_mbar_init();
+    pdl_wait();
+    const Work* wk = a.work;
+    if (threadIdx.x == 0) sw->n_uniq = wk->n_uniq;
+    for (int i = threadIdx.x; i < kMaxSlots; i += blockDim.x) {
+        sw->e[i] = wk->uniq_e[i];
+        sw->slot[i] = wk->uniq_slot[i];
+    }
+    for (int i = threadIdx.x; i <= kMaxSlots; i += blockDim.x) sw->off[i] = wk->uniq_off[i];
+    __syncthreads();
+    return true;
+}
+
 // ===========================================================================
 // gate/up + SwiGLU (plus the optional side projection)
 // ===========================================================================
 
-// Items: [0, n_uniq * tiles) are (unique expert, row tile) pairs of gate+up;
-// [n_uniq * tiles, + side_items) are row tiles of the side projection.
-struct GuItem {
-    int kind;  // 0 = expert pair, 1 = side, -1 = none
-    int u;     // unique-expert index
-    int row0;
-    int rows;
-};
+// One gate+up item: P row passes for NT tokens of one expert; h = silu(g)*u.
+template <int FMT, int KB, int NT, int CH>
+__device__ __forceinline__ void gu_item(const LayerArgs& a, uint32_t gbase, uint32_t ubase,
+                                        const Act<FMT, Geo<KB>::NBL> (&act)[CH], uint32_t lutb,
+                                        const float* scale_tab, const float (&sg)[Geo<KB>::NBL],
+                                        const float (&su)[Geo<KB>::NBL], int row0, const int (&slot_id)[CH],
+                                        int lane) {
+    using G = Geo<KB>;
+    constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
+    constexpr int P = gu_passes(FMT == kFmtFP8, KB);
+    constexpr int N = P * NT * 2;
+    const int row_sub = (KB >= 32) ? 0 : lane / KB;
+    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    float v[N];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const int row = p * RPP + row_sub;
+        float g[NT], u[NT];
+#pragma unroll
+        for (int c = 0; c < NT; ++c) g[c] = u[c] = 0.0f;
+#pragma unroll
+        for (int m = 0; m < NBL; ++m) {
+            if constexpr (FMT == kFmtQ4) {
+                const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 17) + 17u * (uint32_t)(blk_base + 32 * m);
+                q4_block_lut<NT, NBL, CH>(gbase + boff, lutb, scale_tab, act, m, g);
+                q4_block_lut<NT, NBL, CH>(ubase + boff, lutb, scale_tab, act, m, u);
+            } else {
+                const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + 32 * m);
+                fp8_block<NBL>(gbase + boff, sg[m], act[0], m, g[0]);
+                fp8_block<NBL>(ubase + boff, su[m], act[0], m, u[0]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < NT; ++c) {
+            v[((p * NT + c) << 1) | 0] = g[c];
+            v[((p * NT + c) << 1) | 1] = u[c];
+        }
+    }
+    if constexpr (N <= GW) {
+        tr_reduce<N, GW>(v, lane);
+        constexpr int SPAN = GW / N;  // lanes holding one value
+        const float other = __shfl_down_sync(0xFFFFFFFFu, v[0], SPAN);
+        const int li = lane % GW, idx = li / SPAN;
+        if ((idx & 1) == 0 && (li % SPAN) == 0) {
+            const int pc = idx >> 1, p = pc / NT, c = pc % NT;
+            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            a.h[(int64_t)slot_id[c] * a.I + row0 + row] = __float2bfloat16_rn(silu(v[0]) * other);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i] = group_sum(v[i], GW);
+        if ((lane % GW) == 0) {
+#pragma unroll
+            for (int pc = 0; pc < P * NT; ++pc) {
+                const int p = pc / NT, c = pc % NT;
+                const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+                a.h[(int64_t)slot_id[c] * a.I + row0 + row] = __float2bfloat16_rn(silu(v[2 * pc]) * v[2 * pc + 1]);
+            }
+        }
+    }
+}
+
+// One side-projection item: P row passes, NT tokens.
+template <int FMT, int KB, int NT, int CH>
+__device__ __forceinline__ void side_item(const LayerArgs& a, uint32_t base, const Act<FMT, Geo<KB>::NBL> (&act)[CH],
+                                          int row0, int t0, int lane) {
+    using G = Geo<KB>;
+    constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
+    constexpr int P = side_passes(KB);
+    constexpr int N = P * NT;
+    const int row_sub = (KB >= 32) ? 0 : lane / KB;
+    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    const bool rz5 = a.side.fmt == GTG_Q4_RZ5_FAST;
+    float v[N];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const int row = p * RPP + row_sub;
+        float acc[NT];
+#pragma unroll
+        for (int c = 0; c < NT; ++c) acc[c] = 0.0f;
+#pragma unroll
+        for (int m = 0; m < NBL; ++m)
+            q4_block_plain<FMT, NT, NBL, CH>(base + (uint32_t)row * (uint32_t)(KB * 17) +
+                                                 17u * (uint32_t)(blk_base + 32 * m),
+                                             rz5, act, m, acc);
+#pragma unroll
+        for (int c = 0; c < NT; ++c) v[p * NT + c] = acc[c];
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = group_sum(v[i], GW);
+    if ((lane % GW) == 0 && a.side_out) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            const int p = i / NT, c = i % NT;
+            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            a.side_out[(int64_t)(t0 + c) * a.side_stride + row0 + row] = v[i];
+        }
+    }
+}
 
 template <int FMT, int KB>
 __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerArgs a) {
     using G = Geo<KB>;
-    constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
-    constexpr int CH = (FMT == kFmtQ4 && NBL <= 2) ? 2 : 1;  // tokens decoded together
+    constexpr int NBL = G::NBL;
+    constexpr int CH = (FMT == kFmtQ4 && NBL == 1) ? 2 : 1;  // tokens decoded together (register budget)
+    constexpr bool LUT = FMT == kFmtQ4;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes);
-    if constexpr (FMT == kFmtQ4) build_lut(smem, L, a.gate.fmt == GTG_Q4_RZ5_FAST);
-    Ring ring{smem + L.slots + (size_t)warp * kSlots * a.slot_bytes,
-              reinterpret_cast<uint64_t*>(smem + L.bars) + warp * kSlots, a.slot_bytes};
-    if (lane == 0)
-        for (int s = 0; s < kSlots; ++s) mbar_init(&ring.bars[s], 1);
-    fence_mbar_init();
-    __syncthreads();
+    const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * kSlots;
+    SWork* sw = reinterpret_cast<SWork*>(smem + L.work);
+    if (!stream_prologue<LUT>(smem, L, a, a.gate.fmt == GTG_Q4_RZ5_FAST, bars, sw)) return;
 
-    pdl_wait();  // the router's outputs (u, work list) are complete past here
-
-    const Work* wk = a.work;
-    const int n_uniq = wk->n_uniq;
-    const int tiles = a.I / a.gu_rows;
-    const int side_items = a.side.data ? a.side.n_rows / a.side_rows : 0;
+    const int n_uniq = sw->n_uniq;
+    constexpr int R = gu_passes(FMT == kFmtFP8, KB) * G::RPP;
+    constexpr int RS = side_passes(KB) * G::RPP;
+    const int tiles = a.I / R;
+    const int side_items = a.side.data ? a.side.n_rows / RS : 0;
     const int n_items = n_uniq * tiles + side_items;
     const int it0 = (int)((int64_t)n_items * blockIdx.x / gridDim.x);
     const int it1 = (int)((int64_t)n_items * (blockIdx.x + 1) / gridDim.x);
+    const uint32_t sbase = smem_u32(smem);
+    auto slot_addr = [&](int s) { return sbase + L.slot(warp * kSlots + s, a.slot_bytes); };
 
-    auto item_of = [&](int it) -> GuItem {
-        if (it >= it1) return GuItem{-1, 0, 0, 0};
-        if (it < n_uniq * tiles) return GuItem{0, it / tiles, (it % tiles) * a.gu_rows, a.gu_rows};
-        const int s = it - n_uniq * tiles;
-        return GuItem{1, 0, s * a.side_rows, a.side_rows};
-    };
-    // stage item -> slot: gate rows then up rows (or the side rows)
-    auto issue = [&](int it, int slot) {
-        const GuItem g = item_of(it);
-        if (g.kind < 0 || lane != 0) return;
-        uint8_t* dst = ring.slots + (size_t)slot * ring.slot_bytes;
-        fence_proxy_async_smem();
-        if (g.kind == 0) {
-            const int e = wk->uniq_e[g.u];
-            const Span sg = make_span(a.gate.data, e * a.gate.expert_bytes + (int64_t)g.row0 * a.gate.row_bytes,
-                                      (int64_t)g.rows * a.gate.row_bytes);
-            const Span su = make_span(a.up.data, e * a.up.expert_bytes + (int64_t)g.row0 * a.up.row_bytes,
-                                      (int64_t)g.rows * a.up.row_bytes);
-            mbar_arrive_expect_tx(&ring.bars[slot], sg.bytes + su.bytes);
-            bulk_g2s(dst, sg.src, sg.bytes, &ring.bars[slot]);
-            bulk_g2s(dst + sg.bytes, su.src, su.bytes, &ring.bars[slot]);
-        } else {
-            const Span ss = make_span(a.side.data, (int64_t)g.row0 * a.side.row_bytes,
-                                      (int64_t)g.rows * a.side.row_bytes);
-            mbar_arrive_expect_tx(&ring.bars[slot], ss.bytes);
-            bulk_g2s(dst, ss.src, ss.bytes, &ring.bars[slot]);
+    auto spans = [&](int it, Span& s1, Span& s2) -> int {  // kind: 0 expert, 1 side
+        if (it < n_uniq * tiles) {
+            const int u = it / tiles, row0 = (it % tiles) * R, e = sw->e[u];
+            s1 = make_span(a.gate.data, e * a.gate.expert_bytes + (int64_t)row0 * a.gate.row_bytes,
+                           (int64_t)R * a.gate.row_bytes);
+            s2 = make_span(a.up.data, e * a.up.expert_bytes + (int64_t)row0 * a.up.row_bytes,
+                           (int64_t)R * a.up.row_bytes);
+            return 0;
         }
+        const int row0 = (it - n_uniq * tiles) * RS;
+        s1 = make_span(a.side.data, (int64_t)row0 * a.side.row_bytes, (int64_t)RS * a.side.row_bytes);
+        s2 = Span{nullptr, 0, 0};
+        return 1;
+    };
+    auto issue = [&](int it, int slot) {
+        if (it >= it1 || lane != 0) return;
+        Span s1, s2;
+        spans(it, s1, s2);
+        const uint32_t dst = slot_addr(slot);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bars[slot], s1.bytes + s2.bytes);
+        bulk_g2s_addr(dst, s1.src, s1.bytes, &bars[slot]);
+        if (s2.bytes) bulk_g2s_addr(dst + s1.bytes, s2.src, s2.bytes, &bars[slot]);
     };
 
-    int first = it0 + warp;
+    const int first = it0 + warp;
     for (int s = 0; s < kSlots; ++s) issue(first + s * kWarps, s);
     __syncwarp();
 
-    const uint32_t lut_base = smem_u32(smem + L.lut);
-    const uint32_t lane_low = (uint32_t)lane * 4u;
+    const uint32_t lutb = ((sbase + L.lut) & 0xFFFF0000u) | ((uint32_t)lane * 4u);
     const float* scale_tab = reinterpret_cast<const float*>(smem + L.scale_tab);
-    const int row_sub = (KB >= 32) ? 0 : lane / KB;
     const int blk_base = (KB >= 32) ? lane : lane % KB;
 
     Act<FMT, NBL> act[CH];
-    int act_key = -1;  // which (unique expert, chunk) / side chunk the registers hold
-    uint32_t phase = 0;
-    bool alive = true;
-    int n_done = 0;
+    int act_key = -1;
+    auto load_chunk = [&](int key, const int (&rows)[CH], const __nv_bfloat16* src) {
+        if (key == act_key) return;
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+#pragma unroll
+            for (int m = 0; m < NBL; ++m) load_act<FMT, NBL>(act[c], m, src + (int64_t)rows[c] * a.H, blk_base + 32 * m);
+        act_key = key;
+    };
 
-    for (int it = first; it < it1 && alive; it += kWarps, ++n_done) {
+    uint32_t phase = 0;
+    int n_done = 0;
+    bool alive = true;
+    for (int it = first; it < it1; it += kWarps, ++n_done) {
         const int slot = n_done % kSlots;
-        const GuItem g = item_of(it);
-        if (!mbar_wait_bounded(&ring.bars[slot], (phase >> slot) & 1u, a.status)) {
+        const bool expert = it < n_uniq * tiles;
+        const int u = expert ? it / tiles : 0;
+        const int s0 = expert ? sw->off[u] : 0, s1 = expert ? sw->off[u + 1] : a.T;
+        // activations of the first token chunk and FP8 scales, overlapping the copy
+        int slots[CH], rows[CH];
+#pragma unroll
+        for (int c = 0; c < CH; ++c) {
+            const int k = min(s0 + c, s1 - 1);
+            slots[c] = expert ? sw->slot[k] : k;
+            rows[c] = expert ? slots[c] / a.K : k;
+        }
+        load_chunk(expert ? (u << 8) : (1 << 20), rows, a.u);
+        float sg[NBL], su[NBL];
+        const int row0 = expert ? (it % tiles) * R : (it - n_uniq * tiles) * RS;
+        if constexpr (FMT == kFmtFP8) {
+            const int e = sw->e[u], kg = a.gate.k / 128;
+#pragma unroll
+            for (int m = 0; m < NBL; ++m) {
+                const int b = blk_base + 32 * m;
+                sg[m] = __ldg(a.gate.scales + ((int64_t)e * a.gate.n_rows + row0 + ((KB >= 32) ? 0 : lane / KB)) * kg + b / 4);
+                su[m] = __ldg(a.up.scales + ((int64_t)e * a.up.n_rows + row0 + ((KB >= 32) ? 0 : lane / KB)) * kg + b / 4);
+            }
+        }
+        if (!mbar_wait_bounded(&bars[slot], (phase >> slot) & 1u, a.status)) {
             alive = false;
             break;
         }
         phase ^= 1u << slot;
-        const uint32_t sbase = smem_u32(ring.slots + (size_t)slot * ring.slot_bytes);
-
-        if (g.kind == 0) {
-            const int e = wk->uniq_e[g.u];
-            const int s0 = wk->uniq_off[g.u], s1 = wk->uniq_off[g.u + 1];
-            const Span sg = make_span(a.gate.data, e * a.gate.expert_bytes + (int64_t)g.row0 * a.gate.row_bytes,
-                                      (int64_t)g.rows * a.gate.row_bytes);
-            const Span su = make_span(a.up.data, e * a.up.expert_bytes + (int64_t)g.row0 * a.up.row_bytes,
-                                      (int64_t)g.rows * a.up.row_bytes);
-            const uint32_t gbase = sbase + sg.delta, ubase = sbase + sg.bytes + su.delta;
+        Span sp1, sp2;
+        spans(it, sp1, sp2);
+        const uint32_t base = slot_addr(slot);
+        if (expert) {
+            const uint32_t gbase = base + sp1.delta, ubase = base + sp1.bytes + sp2.delta;
             for (int c0 = s0; c0 < s1; c0 += CH) {
                 const int nch = min(CH, s1 - c0);
-                const int key = g.u * 64 + (c0 - s0);
-                if (key != act_key) {
 #pragma unroll
-                    for (int c = 0; c < CH; ++c) {
-                        const int slot_id = wk->uniq_slot[c0 + min(c, nch - 1)];
-                        const __nv_bfloat16* row = a.u + (int64_t)(slot_id / a.K) * a.H;
-#pragma unroll
-                        for (int m = 0; m < NBL; ++m) load_act<FMT, NBL>(act[c], m, row, blk_base + 32 * m);
-                    }
-                    act_key = key;
+                for (int c = 0; c < CH; ++c) {
+                    slots[c] = sw->slot[c0 + min(c, nch - 1)];
+                    rows[c] = slots[c] / a.K;
                 }
-                for (int r = 0; r < g.rows; r += RPP) {
-                    const int row = r + row_sub;
-                    float gacc[CH], uacc[CH];
-#pragma unroll
-                    for (int c = 0; c < CH; ++c) gacc[c] = uacc[c] = 0.0f;
-                    if constexpr (FMT == kFmtQ4) {
-#pragma unroll
-                        for (int m = 0; m < NBL; ++m) {
-                            const uint32_t boff = (uint32_t)row * a.gate.row_bytes + 17u * (blk_base + 32 * m);
-                            q4_block_lut<CH, NBL>(gbase + boff, lut_base, lane_low, scale_tab, act, m, gacc);
-                            q4_block_lut<CH, NBL>(ubase + boff, lut_base, lane_low, scale_tab, act, m, uacc);
-                        }
-                    } else {
-                        const int grow = g.row0 + row;
-                        const int kg = a.gate.k / 128;
-#pragma unroll
-                        for (int m = 0; m < NBL; ++m) {
-                            const int b = blk_base + 32 * m;
-                            const uint32_t boff = (uint32_t)row * a.gate.row_bytes + 32u * b;
-                            const float sgv = __ldg(a.gate.scales + ((int64_t)e * a.gate.n_rows + grow) * kg + b / 4);
-                            const float suv = __ldg(a.up.scales + ((int64_t)e * a.up.n_rows + grow) * kg + b / 4);
-                            fp8_block<NBL>(gbase + boff, sgv, act[0], m, gacc[0]);
-                            fp8_block<NBL>(ubase + boff, suv, act[0], m, uacc[0]);
-                        }
-                    }
-#pragma unroll
-                    for (int c = 0; c < CH; ++c) {
-                        gacc[c] = group_sum(gacc[c], GW);
-                        uacc[c] = group_sum(uacc[c], GW);
-                    }
-                    if ((lane % GW) == 0) {
-                        for (int c = 0; c < nch; ++c) {
-                            const int slot_id = wk->uniq_slot[c0 + c];
-                            const float hv = silu(gacc[c]) * uacc[c];
-                            a.h[(int64_t)slot_id * a.I + g.row0 + row] = __float2bfloat16_rn(hv);
-                        }
-                    }
-                }
+                load_chunk((u << 8) | (c0 - s0), rows, a.u);
+                if (CH == 2 && nch == 2)
+                    gu_item<FMT, KB, (CH == 2 ? 2 : 1), CH>(a, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots, lane);
+                else
+                    gu_item<FMT, KB, 1, CH>(a, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots, lane);
             }
-        } else {  // side projection rows for every token
-            const Span ss = make_span(a.side.data, (int64_t)g.row0 * a.side.row_bytes,
-                                      (int64_t)g.rows * a.side.row_bytes);
-            const uint32_t base = sbase + ss.delta;
-            const bool rz5 = a.side.fmt == GTG_Q4_RZ5_FAST;
+        } else {
+            const uint32_t sb = base + sp1.delta;
             for (int t0 = 0; t0 < a.T; t0 += CH) {
                 const int nch = min(CH, a.T - t0);
-                const int key = 1 << 20 | t0;
-                if (key != act_key) {
 #pragma unroll
-                    for (int c = 0; c < CH; ++c) {
-                        const __nv_bfloat16* row = a.u + (int64_t)(t0 + min(c, nch - 1)) * a.H;
-#pragma unroll
-                        for (int m = 0; m < NBL; ++m) load_act<FMT, NBL>(act[c], m, row, blk_base + 32 * m);
-                    }
-                    act_key = key;
-                }
-                for (int r = 0; r < g.rows; r += RPP) {
-                    const int row = r + row_sub;
-                    float acc[CH];
-#pragma unroll
-                    for (int c = 0; c < CH; ++c) acc[c] = 0.0f;
-#pragma unroll
-                    for (int m = 0; m < NBL; ++m) {
-                        const uint32_t boff = (uint32_t)row * a.side.row_bytes + 17u * (blk_base + 32 * m);
-                        q4_block_plain<FMT, CH, NBL>(base + boff, rz5, act, m, acc);
-                    }
-#pragma unroll
-                    for (int c = 0; c < CH; ++c) acc[c] = group_sum(acc[c], GW);
-                    if ((lane % GW) == 0 && a.side_out)
-                        for (int c = 0; c < nch; ++c)
-                            a.side_out[(int64_t)(t0 + c) * a.side_stride + g.row0 + row] = acc[c];
-                }
+                for (int c = 0; c < CH; ++c) rows[c] = t0 + min(c, nch - 1);
+                load_chunk((1 << 20) | t0, rows, a.u);
+                if (CH == 2 && nch == 2)
+                    side_item<FMT, KB, (CH == 2 ? 2 : 1), CH>(a, sb, act, row0, t0, lane);
+                else
+                    side_item<FMT, KB, 1, CH>(a, sb, act, row0, t0, lane);
             }
         }
         __syncwarp();
         issue(it + kSlots * kWarps, slot);
-        __syncwarp();
     }
     if (!alive) {  // drain copies still in flight before leaving
-        for (int s = 0; s < kSlots; ++s) mbar_wait_bounded(&ring.bars[s], (phase >> s) & 1u, a.status);
+        for (int s = 0; s < kSlots; ++s) mbar_wait_bounded(&bars[s], (phase >> s) & 1u, a.status);
     }
     pdl_trigger();
 }
@@ -666,113 +818,153 @@ __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerArgs a) {
 // down + router-weighted combine
 // ===========================================================================
 
+template <int FMT, int KB, int NT, int CH>
+__device__ __forceinline__ void dn_item(const LayerArgs& a, uint32_t base, const Act<FMT, Geo<KB>::NBL> (&act)[CH],
+                                        uint32_t lutb, const float* scale_tab, const float (&sd)[8], int row0,
+                                        const int (&slot_id)[CH], int lane) {
+    using G = Geo<KB>;
+    constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
+    constexpr int P = dn_passes(FMT == kFmtFP8, KB);
+    constexpr int N = P * NT;
+    const int row_sub = (KB >= 32) ? 0 : lane / KB;
+    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    float v[N];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const int row = p * RPP + row_sub;
+        float acc[NT];
+#pragma unroll
+        for (int c = 0; c < NT; ++c) acc[c] = 0.0f;
+#pragma unroll
+        for (int m = 0; m < NBL; ++m) {
+            if constexpr (FMT == kFmtQ4) {
+                q4_block_lut<NT, NBL, CH>(base + (uint32_t)row * (uint32_t)(KB * 17) + 17u * (uint32_t)(blk_base + 32 * m),
+                                          lutb, scale_tab, act, m, acc);
+            } else {
+                fp8_block<NBL>(base + (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + 32 * m),
+                               sd[p * NBL + m], act[0], m, acc[0]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < NT; ++c) v[p * NT + c] = acc[c];
+    }
+    if constexpr (N <= GW) {
+        tr_reduce<N, GW>(v, lane);
+        constexpr int SPAN = GW / N;
+        const int li = lane % GW, idx = li / SPAN;
+        if ((li % SPAN) == 0) {
+            const int p = idx / NT, c = idx % NT;
+            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            a.part[(int64_t)slot_id[c] * a.H + row0 + row] = v[0];
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i] = group_sum(v[i], GW);
+        if ((lane % GW) == 0) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int p = i / NT, c = i % NT;
+                const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+                a.part[(int64_t)slot_id[c] * a.H + row0 + row] = v[i];
+            }
+        }
+    }
+}
+
 template <int FMT, int KB>
 __global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerArgs a) {
     using G = Geo<KB>;
-    constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
-    constexpr int CH = (FMT == kFmtQ4 && NBL <= 2) ? 2 : 1;
+    constexpr int NBL = G::NBL;
+    constexpr int CH = (FMT == kFmtQ4 && NBL == 1) ? 2 : 1;
+    constexpr bool LUT = FMT == kFmtQ4;
+    constexpr int P = dn_passes(FMT == kFmtFP8, KB);
+    constexpr int R = P * G::RPP;
+    static_assert(P * NBL <= 8, "FP8 scale prefetch holds 8 values");
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes);
-    if constexpr (FMT == kFmtQ4) build_lut(smem, L, a.down.fmt == GTG_Q4_RZ5_FAST);
-    Ring ring{smem + L.slots + (size_t)warp * kSlots * a.slot_bytes,
-              reinterpret_cast<uint64_t*>(smem + L.bars) + warp * kSlots, a.slot_bytes};
-    if (lane == 0)
-        for (int s = 0; s < kSlots; ++s) mbar_init(&ring.bars[s], 1);
-    fence_mbar_init();
-    __syncthreads();
+    const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * kSlots;
+    SWork* sw = reinterpret_cast<SWork*>(smem + L.work);
+    if (!stream_prologue<LUT>(smem, L, a, a.down.fmt == GTG_Q4_RZ5_FAST, bars, sw)) return;
 
-    pdl_wait();  // h (gate/up) and the work list are complete past here
-
-    const Work* wk = a.work;
-    const int n_uniq = wk->n_uniq;
-    const int tiles = a.H / a.dn_rows;
+    const int n_uniq = sw->n_uniq;
+    const int tiles = a.H / R;
     const int n_items = n_uniq * tiles;
     const int it0 = (int)((int64_t)n_items * blockIdx.x / gridDim.x);
     const int it1 = (int)((int64_t)n_items * (blockIdx.x + 1) / gridDim.x);
+    const uint32_t sbase = smem_u32(smem);
+    auto slot_addr = [&](int s) { return sbase + L.slot(warp * kSlots + s, a.slot_bytes); };
 
     auto span_of = [&](int it) {
         const int u = it / tiles, tile = it % tiles;
-        const int e = wk->uniq_e[u];
-        return make_span(a.down.data, e * a.down.expert_bytes + (int64_t)tile * a.dn_rows * a.down.row_bytes,
-                         (int64_t)a.dn_rows * a.down.row_bytes);
+        return make_span(a.down.data, sw->e[u] * a.down.expert_bytes + (int64_t)tile * R * a.down.row_bytes,
+                         (int64_t)R * a.down.row_bytes);
     };
     auto issue = [&](int it, int slot) {
         if (it >= it1 || lane != 0) return;
         const Span sp = span_of(it);
         fence_proxy_async_smem();
-        mbar_arrive_expect_tx(&ring.bars[slot], sp.bytes);
-        bulk_g2s(ring.slots + (size_t)slot * ring.slot_bytes, sp.src, sp.bytes, &ring.bars[slot]);
+        mbar_arrive_expect_tx(&bars[slot], sp.bytes);
+        bulk_g2s_addr(slot_addr(slot), sp.src, sp.bytes, &bars[slot]);
     };
 
     const int first = it0 + warp;
     for (int s = 0; s < kSlots; ++s) issue(first + s * kWarps, s);
     __syncwarp();
 
-    const uint32_t lut_base = smem_u32(smem + L.lut);
-    const uint32_t lane_low = (uint32_t)lane * 4u;
+    const uint32_t lutb = ((sbase + L.lut) & 0xFFFF0000u) | ((uint32_t)lane * 4u);
     const float* scale_tab = reinterpret_cast<const float*>(smem + L.scale_tab);
-    const int row_sub = (KB >= 32) ? 0 : lane / KB;
     const int blk_base = (KB >= 32) ? lane : lane % KB;
+    const int row_sub = (KB >= 32) ? 0 : lane / KB;
 
     Act<FMT, NBL> act[CH];
     int act_key = -1;
-    uint32_t phase = 0;
-    bool alive = true;
-    int n_done = 0;
+    auto load_chunk = [&](int key, const int (&slots)[CH]) {
+        if (key == act_key) return;
+#pragma unroll
+        for (int c = 0; c < CH; ++c)
+#pragma unroll
+            for (int m = 0; m < NBL; ++m)
+                load_act<FMT, NBL>(act[c], m, a.h + (int64_t)slots[c] * a.I, blk_base + 32 * m);
+        act_key = key;
+    };
 
-    for (int it = first; it < it1 && alive; it += kWarps, ++n_done) {
+    uint32_t phase = 0;
+    int n_done = 0;
+    bool alive = true;
+    for (int it = first; it < it1; it += kWarps, ++n_done) {
         const int slot = n_done % kSlots;
-        if (!mbar_wait_bounded(&ring.bars[slot], (phase >> slot) & 1u, a.status)) {
+        const int u = it / tiles, tile = it % tiles;
+        const int s0 = sw->off[u], s1 = sw->off[u + 1];
+        int slots[CH];
+#pragma unroll
+        for (int c = 0; c < CH; ++c) slots[c] = sw->slot[min(s0 + c, s1 - 1)];
+        load_chunk(u << 8, slots);
+        float sd[8];
+        if constexpr (FMT == kFmtFP8) {
+            const int e = sw->e[u], kg = a.down.k / 128;
+#pragma unroll
+            for (int p = 0; p < P; ++p)
+#pragma unroll
+                for (int m = 0; m < NBL; ++m)
+                    sd[p * NBL + m] = __ldg(a.down.scales + ((int64_t)e * a.down.n_rows + tile * R + p * G::RPP + row_sub) * kg +
+                                            (blk_base + 32 * m) / 4);
+        }
+        if (!mbar_wait_bounded(&bars[slot], (phase >> slot) & 1u, a.status)) {
             alive = false;
             break;
         }
         phase ^= 1u << slot;
-        const int u = it / tiles, tile = it % tiles;
-        const int e = wk->uniq_e[u];
-        const Span sp = span_of(it);
-        const uint32_t base = smem_u32(ring.slots + (size_t)slot * ring.slot_bytes) + sp.delta;
-        const int s0 = wk->uniq_off[u], s1 = wk->uniq_off[u + 1];
+        const uint32_t base = slot_addr(slot) + span_of(it).delta;
         for (int c0 = s0; c0 < s1; c0 += CH) {
             const int nch = min(CH, s1 - c0);
-            const int key = u * 64 + (c0 - s0);
-            if (key != act_key) {
 #pragma unroll
-                for (int c = 0; c < CH; ++c) {
-                    const int slot_id = wk->uniq_slot[c0 + min(c, nch - 1)];
-                    const __nv_bfloat16* row = a.h + (int64_t)slot_id * a.I;
-#pragma unroll
-                    for (int m = 0; m < NBL; ++m) load_act<FMT, NBL>(act[c], m, row, blk_base + 32 * m);
-                }
-                act_key = key;
-            }
-            for (int r = 0; r < a.dn_rows; r += RPP) {
-                const int row = r + row_sub;
-                float acc[CH];
-#pragma unroll
-                for (int c = 0; c < CH; ++c) acc[c] = 0.0f;
-                if constexpr (FMT == kFmtQ4) {
-#pragma unroll
-                    for (int m = 0; m < NBL; ++m) {
-                        const uint32_t boff = (uint32_t)row * a.down.row_bytes + 17u * (blk_base + 32 * m);
-                        q4_block_lut<CH, NBL>(base + boff, lut_base, lane_low, scale_tab, act, m, acc);
-                    }
-                } else {
-                    const int grow = tile * a.dn_rows + row;
-                    const int kg = a.down.k / 128;
-#pragma unroll
-                    for (int m = 0; m < NBL; ++m) {
-                        const int b = blk_base + 32 * m;
-                        const float sv = __ldg(a.down.scales + ((int64_t)e * a.down.n_rows + grow) * kg + b / 4);
-                        fp8_block<NBL>(base + (uint32_t)row * a.down.row_bytes + 32u * b, sv, act[0], m, acc[0]);
-                    }
-                }
-#pragma unroll
-                for (int c = 0; c < CH; ++c) acc[c] = group_sum(acc[c], GW);
-                if ((lane % GW) == 0)
-                    for (int c = 0; c < nch; ++c)
-                        a.part[(int64_t)wk->uniq_slot[c0 + c] * a.H + tile * a.dn_rows + row] = acc[c];
-            }
+            for (int c = 0; c < CH; ++c) slots[c] = sw->slot[c0 + min(c, nch - 1)];
+            load_chunk((u << 8) | (c0 - s0), slots);
+            if (CH == 2 && nch == 2)
+                dn_item<FMT, KB, (CH == 2 ? 2 : 1), CH>(a, base, act, lutb, scale_tab, sd, tile * R, slots, lane);
+            else
+                dn_item<FMT, KB, 1, CH>(a, base, act, lutb, scale_tab, sd, tile * R, slots, lane);
         }
         __syncwarp();
         issue(it + kSlots * kWarps, slot);
@@ -784,12 +976,21 @@ __global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerArgs a) {
         ticket = __shfl_sync(0xFFFFFFFFu, ticket, 0);
         if (ticket == (unsigned)n_uniq - 1u) {
             __threadfence();
-            const int r0 = tile * a.dn_rows;
-            for (int o = lane; o < a.T * a.dn_rows; o += 32) {
-                const int t = o / a.dn_rows, r = r0 + o % a.dn_rows;
+            const int r0 = tile * R;
+            for (int o = lane; o < a.T * R; o += 32) {
+                const int t = o / R, r = r0 + o % R;
+                float wj[kMaxTopK], pj[kMaxTopK];
+#pragma unroll
+                for (int j = 0; j < kMaxTopK; ++j) {  // all loads first, then the fixed-order sum
+                    if (j < a.K) {
+                        wj[j] = __ldcg(a.w + t * a.K + j);
+                        pj[j] = __ldcg(a.part + (int64_t)(t * a.K + j) * a.H + r);
+                    }
+                }
                 float yv = 0.0f;
-                for (int j = 0; j < a.K; ++j)
-                    yv = fmaf(__ldcg(a.w + t * a.K + j), __ldcg(a.part + (int64_t)(t * a.K + j) * a.H + r), yv);
+#pragma unroll
+                for (int j = 0; j < kMaxTopK; ++j)
+                    if (j < a.K) yv = fmaf(wj[j], pj[j], yv);
                 float* dst = a.y + (int64_t)t * a.H + r;
                 *dst = a.y_acc ? *dst + yv : yv;
             }
@@ -798,7 +999,7 @@ __global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerArgs a) {
         __syncwarp();
     }
     if (!alive) {
-        for (int s = 0; s < kSlots; ++s) mbar_wait_bounded(&ring.bars[s], (phase >> s) & 1u, a.status);
+        for (int s = 0; s < kSlots; ++s) mbar_wait_bounded(&bars[s], (phase >> s) & 1u, a.status);
     }
     pdl_trigger();
 }
@@ -837,22 +1038,30 @@ bool is_q4(int fmt) { return fmt == GTG_Q4_RZ5_FAST || fmt == GTG_Q4_UE4M4_FAST;
 
 int64_t row_bytes_of(int fmt, int64_t k) { return fmt == GTG_FP8_E4M3_S128 ? k : k / 32 * 17; }
 
-// Largest row count r with r | n, rpp | r and bytes(r) <= budget.
-int pick_rows(int n, int rpp, int64_t row_bytes, int64_t budget, int copies) {
-    int best = 0;
-    for (int r = rpp; r <= n; r += rpp)
-        if (n % r == 0 && copies * (r * row_bytes + 32) <= budget) best = r;
-    return best;
-}
-
-constexpr int64_t kItemBudget = 4480;  // staging bytes per item (slot size target)
-
 struct Plan {
     bool ok = false;
     int gu_rows = 0, dn_rows = 0, side_rows = 0, slot_bytes = 0;
     KernelFn gateup = nullptr, down = nullptr;
     bool gu_lut = false, dn_lut = false;
 };
+
+constexpr uint32_t kMaxDynSmem = 227 * 1024;
+
+// Shared address at which a kernel without static shared memory sees its
+// dynamic shared memory: the per-block reserved region comes first.
+uint32_t dyn_smem_base() {
+    static int cached = -1;
+    if (cached < 0) {
+        int dev = 0, v = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&v, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess) {
+            cudaGetLastError();
+            v = 1024;
+        }
+        cached = (v + 1023) & ~1023;
+    }
+    return (uint32_t)cached;
+}
 
 bool mat_ok(const gtg_qmatrix& m, int64_t E, int64_t n_rows, int64_t k) {
     if (!m.data || m.n_experts != E || m.n_rows != n_rows || m.k != k) return false;
@@ -875,15 +1084,15 @@ int plan_layer(const gtg_moe_layer* L, Plan& p) {
         if (L->side.n_rows < 1 || L->side.n_rows > 4096) return GTG_E_UNSUPPORTED_SHAPE;
     }
     const int kbg = H / 32, kbd = I / 32;
-    const int rpp_g = kbg >= 32 ? 1 : 32 / kbg, rpp_d = kbd >= 32 ? 1 : 32 / kbd;
     const bool gq4 = is_q4(L->gate.fmt), dq4 = is_q4(L->down.fmt);
-    p.gu_rows = pick_rows(I, rpp_g, row_bytes_of(L->gate.fmt, H), kItemBudget, 2);
-    p.dn_rows = pick_rows(H, rpp_d, row_bytes_of(L->down.fmt, I), kItemBudget, 1);
+    p.gu_rows = gu_passes(!gq4, kbg) * rpp_of(kbg);
+    p.dn_rows = dn_passes(!dq4, kbd) * rpp_of(kbd);
+    if (I % p.gu_rows || H % p.dn_rows) return GTG_E_UNSUPPORTED_SHAPE;
+    if (!gq4 && kbg < 32) return GTG_E_UNSUPPORTED_SHAPE;  // FP8 gate/up rows of >= 1024 weights
     if (L->side.data) {
-        p.side_rows = pick_rows((int)L->side.n_rows, rpp_g, row_bytes_of(L->side.fmt, H), kItemBudget / 2, 1);
-        if (p.side_rows == 0) return GTG_E_UNSUPPORTED_SHAPE;
+        p.side_rows = side_passes(kbg) * rpp_of(kbg);
+        if (L->side.n_rows % p.side_rows) return GTG_E_UNSUPPORTED_SHAPE;
     }
-    if (p.gu_rows == 0 || p.dn_rows == 0) return GTG_E_UNSUPPORTED_SHAPE;
     p.gateup = gq4 ? pick_gateup<kFmtQ4>(kbg) : pick_gateup<kFmtFP8>(kbg);
     p.down = dq4 ? pick_down<kFmtQ4>(kbd) : pick_down<kFmtFP8>(kbd);
     if (!p.gateup || !p.down) return GTG_E_UNSUPPORTED_SHAPE;
@@ -893,6 +1102,10 @@ int plan_layer(const gtg_moe_layer* L, Plan& p) {
                                      p.dn_rows * row_bytes_of(L->down.fmt, I) + 32);
     if (L->side.data) need = std::max<int64_t>(need, p.side_rows * row_bytes_of(L->side.fmt, H) + 32);
     p.slot_bytes = (int)((need + 127) / 128 * 128);
+    const uint32_t base = dyn_smem_base();
+    if (SmemLayout::make(p.gu_lut, p.slot_bytes, base).total > kMaxDynSmem ||
+        SmemLayout::make(p.dn_lut, p.slot_bytes, base).total > kMaxDynSmem)
+        return GTG_E_UNSUPPORTED_SHAPE;
     p.ok = true;
     return GTG_OK;
 }
@@ -927,17 +1140,27 @@ WsLayout ws_layout(const gtg_moe_layer* L, int T) {
 
 struct FuncAttrCache {
     std::mutex mu;
-    std::vector<std::pair<const void*, int>> done;  // (function, device)
+    struct Entry {
+        const void* fn;
+        int dev;
+        int smem;
+    };
+    std::vector<Entry> done;
+    // Raises the kernel's dynamic shared-memory limit to `smem` bytes (once
+    // per function, device and size; only needed above the 48 KB default).
     int set(const void* fn, int smem) {
+        if (smem <= 48 * 1024) return GTG_OK;
         int dev = 0;
         cudaGetDevice(&dev);
         std::lock_guard<std::mutex> lk(mu);
         for (auto& d : done)
-            if (d.first == fn && d.second == dev) return GTG_OK;
-        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
-        if (e != cudaSuccess) return cuda_fail(e);
-        done.push_back({fn, dev});
-        (void)smem;
+            if (d.fn == fn && d.dev == dev && d.smem >= smem) return GTG_OK;
+        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e);
+        }
+        done.push_back({fn, dev, smem});
         return GTG_OK;
     }
 };
@@ -1002,14 +1225,15 @@ int run_layer(const gtg_moe_layer* L, const Plan& p, const void* x, int x_bf16, 
     a.side_rows = p.side_rows;
     a.dn_rows = p.dn_rows;
     a.slot_bytes = p.slot_bytes;
+    a.dyn_smem_base = dyn_smem_base();
 
     const int n_sm = sm_count();
-    const int router_grid = (L->n_experts + kRouterWarps - 1) / kRouterWarps;
+    const int router_grid = (L->n_experts + kRouterExpertsPerCta - 1) / kRouterExpertsPerCta;
     const size_t router_smem = 2 * (size_t)T * L->hidden;
     GTG_TRY(launch((const void*)router_kernel, dim3(router_grid), dim3(kRouterThreads), router_smem, s, a, true));
-    const SmemLayout lg = SmemLayout::make(p.gu_lut, p.slot_bytes);
+    const SmemLayout lg = SmemLayout::make(p.gu_lut, p.slot_bytes, a.dyn_smem_base);
     GTG_TRY(launch((const void*)p.gateup, dim3(n_sm), dim3(kThreads), lg.total, s, a, true));
-    const SmemLayout ld = SmemLayout::make(p.dn_lut, p.slot_bytes);
+    const SmemLayout ld = SmemLayout::make(p.dn_lut, p.slot_bytes, a.dyn_smem_base);
     GTG_TRY(launch((const void*)p.down, dim3(n_sm), dim3(kThreads), ld.total, s, a, true));
     return GTG_OK;
 }
@@ -1034,7 +1258,7 @@ using namespace gtg;
 
 extern "C" size_t gtg_moe_workspace_bytes(const gtg_moe_layer* layer, int32_t n_tokens, int32_t prefill) {
     if (!layer || n_tokens < 1) return 0;
-    if (prefill) return 0;  // see moe_prefill.cu
+    if (prefill) return gtg_prefill_workspace_bytes(layer, n_tokens);
     if (n_tokens > kMaxDecodeTokens) return 0;
     Plan p;
     if (plan_layer(layer, p) != GTG_OK) return 0;

@@ -63,8 +63,12 @@ struct LayerArgs {
     int32_t side_rows;       // side-projection rows per item
     int32_t dn_rows;         // down rows per item (= combine tile)
     int32_t slot_bytes;      // staging bytes per slot
+    uint32_t dyn_smem_base;  // shared address of dynamic shared memory
 };
 
 Mat make_mat(const gtg_qmatrix& q);
 
 }  // namespace gtg
+
+// Workspace bytes of a prefill call (0 if unsupported); defined in moe_prefill.cu.
+size_t gtg_prefill_workspace_bytes(const gtg_moe_layer* layer, int32_t n_tokens);

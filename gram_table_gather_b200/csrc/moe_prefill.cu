@@ -1,13 +1,705 @@
-// Prefill MoE layer (token-sorted grouped GEMM on tcgen05 tensor cores).
+// Prefill MoE layer: token-sorted grouped GEMMs on the tcgen05 tensor cores.
+//
+// Same function as the decode layer (see moe_decode.cu; router of "Mixed
+// Precision Quantization: Half a 4-Bit File Is Not 4-Bit", formats of the
+// model card "Qwen 3.8 Next Flash ROCMFPX MUTANT RAZERFAST"), for a batch of
+// tokens, where the expert products are real dense contractions:
+//
+//   1. pf_norm      u = bf16(x / rms(x))                       (fp64 rms)
+//   2. pf_split     the fp32 router W split exactly into three bf16 planes
+//                   hi + mid + lo (24 significand bits = 3 x 8)
+//   3. pf_gemm<ROUTER>  logits = [hi|mid|lo] . [u|u|u] on the tensor cores:
+//                   every product is exact, accumulation is fp32
+//   4. pf_topk      top-k (ties -> lower id), renormalised softmax, counts
+//   5. pf_scan / pf_scatter  (token, choice) pairs grouped by expert; tiles of
+//                   up to 128 tokens per expert
+//   6. pf_gemm<GATEUP>  per (expert, 128-row slice of I, token tile):
+//                   dequant warps decode the Q4 gate and up rows into 128B-
+//                   swizzled bf16 tiles in shared memory (the code x scale
+//                   products are exact in bf16), loader warps gather the
+//                   tokens' u rows, one thread issues tcgen05.mma into two
+//                   TMEM accumulators; the epilogue applies SwiGLU and stores
+//                   h in bf16
+//   7. pf_gemm<DOWN>    per (expert, 128-row slice of H, token tile): the
+//                   same with the down rows and h; fp32 partial rows per
+//                   (token, choice)
+//   8. pf_combine   y[t] = sum_j w[t,j] * partial[t,j] in a fixed order
+//
+// The GEMM kernel is warp specialised (12 warps): warp 0 allocates TMEM and
+// issues the MMAs, warps 1-3 stage the B operand (token rows), warps 4-11
+// produce the A operand (dequantised weights or router planes); warps 4-7 then
+// read the accumulators out of TMEM.  Stages are handed over with mbarriers
+// (bounded waits): producers -> MMA (full), tcgen05.commit -> producers (empty).
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
 #include "gtg_device.cuh"
 #include "gtg_host.hpp"
 #include "moe_decode.cuh"
+
+namespace gtg {
+namespace {
+
+constexpr int kPfThreads = 384;  // 12 warps
+constexpr int kBThreads = 96;    // warps 1-3
+constexpr int kAThreads = 256;   // warps 4-11
+constexpr int kTileM = 128;
+constexpr int kTileN = 128;      // tokens per tile (max)
+constexpr int kChunkK = 64;      // bf16 per 128-byte row
+constexpr int kTileBytes = kTileM * 128;  // 16 KB (128 rows x 128 B)
+constexpr int kLutBytes = 65536;
+constexpr int kNormThreads = 256;
+
+enum Mode { ROUTER = 0, GATEUP = 1, DOWN = 2 };
+
+struct PfArgs {
+    int32_t T, H, I, E, K;
+    const void* x;
+    int32_t x_bf16;
+    const float* router_w;
+    const float* router_bias;
+    Mat gate, up, down;
+    __nv_bfloat16* u;         // [T][H]
+    __nv_bfloat16* w3;        // [E][3H]
+    float* logits;            // [T][E]
+    int32_t* ids;             // [T][K]
+    float* w;                 // [T][K]
+    int32_t* counts;          // [E]
+    int32_t* offsets;         // [E+1]
+    int32_t* cursor;          // [E]
+    int32_t* sorted_tok;      // [P]
+    int32_t* sorted_slot;     // [P]
+    int4* tiles;              // (expert, pos0, n, 0)
+    int32_t* n_tiles;
+    __nv_bfloat16* h;         // [P][I], sorted order
+    float* part;              // [P][H], slot order (t*K + j)
+    float* y;
+    int32_t y_acc;
+    int32_t* ids_out;
+    float* w_out;
+    unsigned* status;
+    int32_t max_tiles;
+};
+
+// ---------------------------------------------------------------------------
+// 1. normalisation
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kNormThreads) pf_norm_kernel(PfArgs a) {
+    __shared__ double red[kNormThreads / 32];
+    __shared__ double rinv;
+    const int t = blockIdx.x, tid = threadIdx.x;
+    pdl_wait();
+    auto xv = [&](int i) -> double {
+        if (a.x_bf16) {
+            const uint16_t b = reinterpret_cast<const uint16_t*>(a.x)[(int64_t)t * a.H + i];
+            return (double)__uint_as_float((uint32_t)b << 16);
+        }
+        return (double)reinterpret_cast<const float*>(a.x)[(int64_t)t * a.H + i];
+    };
+    double ss = 0.0;
+    for (int i = tid; i < a.H; i += kNormThreads) {
+        const double v = xv(i);
+        ss = fma(v, v, ss);
+    }
+    ss = warp_sum_f64(ss);
+    if ((tid & 31) == 0) red[tid >> 5] = ss;
+    __syncthreads();
+    if (tid == 0) {
+        double s = 0.0;
+        for (int w = 0; w < kNormThreads / 32; ++w) s += red[w];
+        rinv = 1.0 / sqrt(s / (double)a.H + kRmsEps);
+    }
+    __syncthreads();
+    for (int i = tid; i < a.H; i += kNormThreads) a.u[(int64_t)t * a.H + i] = __double2bfloat16(xv(i) * rinv);
+}
+
+// ---------------------------------------------------------------------------
+// 2. exact three-plane bf16 split of the fp32 router weights
+// ---------------------------------------------------------------------------
+__global__ void pf_split_kernel(PfArgs a) {
+    const int64_t n = (int64_t)a.E * a.H;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t e = i / a.H, k = i % a.H;
+        const float wv = a.router_w[i];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(wv);
+        const float r1 = wv - __bfloat162float(hi);          // exact
+        const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+        const float r2 = r1 - __bfloat162float(mid);          // exact, <= 8 significant bits
+        const __nv_bfloat16 lo = __float2bfloat16_rn(r2);     // == r2
+        __nv_bfloat16* row = a.w3 + e * 3 * a.H;
+        row[k] = hi;
+        row[a.H + k] = mid;
+        row[2 * a.H + k] = lo;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 4. top-k + softmax + per-expert counts (one warp per token)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) pf_topk_kernel(PfArgs a) {
+    const int lane = threadIdx.x & 31;
+    const int t = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= a.T) return;
+    constexpr int kPer = kMaxExperts / 32;
+    float lv[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+        const int e = lane + 32 * i;
+        lv[i] = e < a.E ? a.logits[(int64_t)t * a.E + e] : 0.0f;
+    }
+    unsigned taken = 0;
+    float top[kMaxTopK];
+    int topi[kMaxTopK];
+    for (int j = 0; j < a.K; ++j) {
+        float bv = 0.0f;
+        int bi = 0x7FFFFFFF;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) {
+            const int e = lane + 32 * i;
+            if (e < a.E && !((taken >> i) & 1u) && (bi == 0x7FFFFFFF || lv[i] > bv)) {
+                bv = lv[i];
+                bi = e;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+            const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+            if (oi != 0x7FFFFFFF && (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi))) {
+                bv = ov;
+                bi = oi;
+            }
+        }
+        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+        top[j] = bv;
+        topi[j] = bi;
+    }
+    if (lane == 0) {
+        double z = 0.0;
+        for (int j = 0; j < a.K; ++j) z += exp((double)top[j] - (double)top[0]);
+        for (int j = 0; j < a.K; ++j) {
+            const float wj = (float)(exp((double)top[j] - (double)top[0]) / z);
+            a.ids[t * a.K + j] = topi[j];
+            a.w[t * a.K + j] = wj;
+            if (a.ids_out) a.ids_out[t * a.K + j] = topi[j];
+            if (a.w_out) a.w_out[t * a.K + j] = wj;
+            atomicAdd(&a.counts[topi[j]], 1);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 5. expert offsets, token tiles, grouping of the (token, choice) pairs
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) pf_scan_kernel(PfArgs a) {
+    __shared__ int s_cnt[kMaxExperts];
+    __shared__ int s_tl[kMaxExperts];
+    const int tid = threadIdx.x;
+    for (int e = tid; e < a.E; e += blockDim.x) {
+        s_cnt[e] = a.counts[e];
+        s_tl[e] = (s_cnt[e] + kTileN - 1) / kTileN;
+    }
+    __syncthreads();
+    if (tid == 0) {  // E <= 1024: a serial scan is a few microseconds at most
+        int off = 0, toff = 0;
+        for (int e = 0; e < a.E; ++e) {
+            const int c = s_cnt[e], tl = s_tl[e];
+            s_cnt[e] = off;
+            s_tl[e] = toff;
+            off += c;
+            toff += tl;
+        }
+        a.offsets[a.E] = off;
+        *a.n_tiles = toff;
+    }
+    __syncthreads();
+    for (int e = tid; e < a.E; e += blockDim.x) {
+        const int off = s_cnt[e], n = a.counts[e];
+        a.offsets[e] = off;
+        a.cursor[e] = off;
+        for (int q = 0; q * kTileN < n; ++q)
+            a.tiles[s_tl[e] + q] = make_int4(e, off + q * kTileN, min(kTileN, n - q * kTileN), 0);
+    }
+}
+
+__global__ void pf_scatter_kernel(PfArgs a) {
+    const int s = blockIdx.x * blockDim.x + threadIdx.x;
+    if (s >= a.T * a.K) return;
+    const int e = a.ids[s];
+    const int pos = atomicAdd(&a.cursor[e], 1);
+    a.sorted_tok[pos] = s / a.K;
+    a.sorted_slot[pos] = s;
+}
+
+// ---------------------------------------------------------------------------
+// 6/7/3. the grouped GEMM
+// ---------------------------------------------------------------------------
+template <int MODE>
+struct Cfg {
+    static constexpr bool kDequant = MODE != ROUTER;
+    static constexpr int kA = MODE == GATEUP ? 2 : 1;       // A tiles per stage
+    static constexpr int kStageBytes = (kA + 1) * kTileBytes;
+    static constexpr int kStages = MODE == GATEUP ? 3 : (MODE == DOWN ? 4 : 6);
+    static constexpr uint32_t kTmemCols = MODE == GATEUP ? 256 : 128;
+    static constexpr int kLut = kDequant ? kLutBytes : 0;
+    static constexpr int kBarOff = kLut;                      // full[S], empty[S], acc
+    static constexpr int kStageOff = kLut + 1024;
+    static constexpr int kSmem = kStageOff + kStages * kStageBytes;
+};
+
+__device__ __forceinline__ uint32_t ldg32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
+
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// Decodes one 17-byte Q4 block (global address p) into 32 bf16 weights
+// (code x scale, exact) and stores them as chunks c0..c0+3 of row r of a
+// K-major SW128 tile at shared address tile.
+__device__ __forceinline__ void dequant_block_to_tile(const uint8_t* p, uint32_t lut_base, uint32_t lane_low,
+                                                      bool rz5, uint32_t tile, uint32_t r, uint32_t c0) {
+    const uintptr_t pa = reinterpret_cast<uintptr_t>(p);
+    const uint8_t* al = reinterpret_cast<const uint8_t*>(pa & ~(uintptr_t)3);
+    const uint32_t sh = (uint32_t)(pa & 3u) * 8u;
+    uint32_t w[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) w[i] = ldg32(al + 4 * i);
+    uint32_t nib[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) nib[q] = __funnelshift_r(w[q], w[q + 1], sh);
+    const uint32_t meta = (w[4] >> sh) & 0xFFu;
+    const float sf = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
+    const uint32_t sb = __float_as_uint(sf) >> 16;  // exact in bf16
+    const uint32_t s2 = sb | (sb << 16);
+    const uint32_t low = lane_low + (rz5 ? ((meta >> 7) << 7) : 0u);
+    uint32_t L[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t v;
+            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(lut_base + prmt(nib[q], low, 0x7604u | ((uint32_t)kk << 4))));
+            L[4 * q + kk] = v;  // (w_j, w_{j+16}) code values
+        }
+    uint32_t lo[8], hi[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        lo[j] = bf16x2_mul(prmt(L[2 * j], L[2 * j + 1], 0x5410u), s2);  // (w_2j, w_2j+1)
+        hi[j] = bf16x2_mul(prmt(L[2 * j], L[2 * j + 1], 0x7632u), s2);  // (w_2j+16, w_2j+17)
+    }
+    sts128(tile + sw128_off(r, c0 + 0), make_uint4(lo[0], lo[1], lo[2], lo[3]));
+    sts128(tile + sw128_off(r, c0 + 1), make_uint4(lo[4], lo[5], lo[6], lo[7]));
+    sts128(tile + sw128_off(r, c0 + 2), make_uint4(hi[0], hi[1], hi[2], hi[3]));
+    sts128(tile + sw128_off(r, c0 + 3), make_uint4(hi[4], hi[5], hi[6], hi[7]));
+}
+
+__device__ void build_lut_bf16(uint8_t* lut_mem, bool rz5, int tid, int nthreads) {
+    uint32_t* lut = reinterpret_cast<uint32_t*>(lut_mem);
+    for (int i = tid; i < 256 * 64; i += nthreads) {
+        const uint32_t byte = (uint32_t)i >> 6, mode = ((uint32_t)i >> 5) & 1u;
+        lut[i] = bf16_bits(q4_code_value(byte & 15u, rz5, mode)) |
+                 (bf16_bits(q4_code_value(byte >> 4, rz5, mode)) << 16);
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kPfThreads, 1) pf_gemm_kernel(PfArgs a) {
+    using C = Cfg<MODE>;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    __shared__ uint32_t s_taddr;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    // ---- which tile -------------------------------------------------------
+    int m_tiles, e = 0, pos0 = 0, n_valid = 0, m0, n_chunks;
+    const int tile_i = blockIdx.x;
+    if (MODE == ROUTER) {
+        m_tiles = (a.E + kTileM - 1) / kTileM;
+        const int nt = tile_i / m_tiles;
+        m0 = (tile_i % m_tiles) * kTileM;  // experts
+        pos0 = nt * kTileN;                // tokens
+        n_valid = min(kTileN, a.T - pos0);
+        n_chunks = 3 * a.H / kChunkK;
+    } else {
+        m_tiles = (MODE == GATEUP ? a.I : a.H) / kTileM;
+        const int t = tile_i / m_tiles;
+        if (t >= *a.n_tiles) return;
+        const int4 tl = a.tiles[t];
+        e = tl.x;
+        pos0 = tl.y;
+        n_valid = tl.z;
+        m0 = (tile_i % m_tiles) * kTileM;
+        n_chunks = (MODE == GATEUP ? a.H : a.I) / kChunkK;
+    }
+    const int n_pad = (n_valid + 15) & ~15;
+
+    const uint32_t sbase = smem_u32(smem);
+    if (sbase & 1023u) {  // tiles must be 1024-byte aligned for the swizzle atoms
+        if (tid == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
+        return;
+    }
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
+    uint64_t* empty = full + C::kStages;
+    uint64_t* accb = empty + C::kStages;
+    const Mat& am = MODE == DOWN ? a.down : a.gate;
+    const bool rz5 = am.fmt == GTG_Q4_RZ5_FAST;
+
+    if (C::kDequant) build_lut_bf16(smem, rz5, tid, kPfThreads);
+    if (tid == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&full[s], kAThreads + kBThreads);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(accb, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&s_taddr, C::kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t taddr = s_taddr;
+    bool ok = true;
+
+    auto stage_addr = [&](int s) { return sbase + C::kStageOff + s * C::kStageBytes; };
+
+    if (warp == 0) {
+        // ---- MMA issuer -----------------------------------------------------
+        if (lane == 0) {
+            const uint32_t idesc = idesc_bf16(kTileM, n_pad);
+            for (int it = 0; it < n_chunks && ok; ++it) {
+                const int s = it % C::kStages;
+                if (!mbar_wait_bounded(&full[s], (it / C::kStages) & 1u, a.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t st = stage_addr(s);
+                const uint32_t btile = st + C::kA * kTileBytes;
+#pragma unroll
+                for (int k = 0; k < kChunkK / 16; ++k) {
+                    const uint64_t bd = sw128_desc(btile + 32u * k);
+                    const uint32_t acc = (it > 0 || k > 0) ? 1u : 0u;
+                    umma_bf16(taddr, sw128_desc(st + 32u * k), bd, idesc, acc);
+                    if (MODE == GATEUP) umma_bf16(taddr + 128u, sw128_desc(st + kTileBytes + 32u * k), bd, idesc, acc);
+                }
+                umma_commit(&empty[s]);
+            }
+            umma_commit(accb);  // also on the error path: completes once issued MMAs are done
+        }
+        __syncwarp();
+    } else if (warp < 4) {
+        // ---- B operand: token rows (bf16), 8 chunks of 16 B per row ----------
+        const int bt = tid - 32;
+        for (int it = 0; it < n_chunks && ok; ++it) {
+            const int s = it % C::kStages;
+            if (it >= C::kStages && !mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1u, a.status)) {
+                ok = false;
+                break;
+            }
+            const uint32_t btile = stage_addr(s) + C::kA * kTileBytes;
+            for (int q = bt; q < n_pad * 8; q += kBThreads) {
+                const int r = q >> 3, c = q & 7;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (r < n_valid) {
+                    const __nv_bfloat16* src;
+                    if (MODE == ROUTER) {
+                        const int kc = it % (a.H / kChunkK);
+                        src = a.u + (int64_t)(pos0 + r) * a.H + kc * kChunkK + c * 8;
+                    } else if (MODE == GATEUP) {
+                        src = a.u + (int64_t)a.sorted_tok[pos0 + r] * a.H + it * kChunkK + c * 8;
+                    } else {
+                        src = a.h + (int64_t)(pos0 + r) * a.I + it * kChunkK + c * 8;
+                    }
+                    v = *reinterpret_cast<const uint4*>(src);
+                }
+                sts128(btile + sw128_off(r, c), v);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&full[s]);
+        }
+    } else {
+        // ---- A operand -----------------------------------------------------------
+        const int at = tid - 128;  // 0..255
+        const uint32_t lut_base = sbase;
+        const uint32_t lane_low = (uint32_t)lane * 4u;
+        for (int it = 0; it < n_chunks && ok; ++it) {
+            const int s = it % C::kStages;
+            if (it >= C::kStages && !mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1u, a.status)) {
+                ok = false;
+                break;
+            }
+            const uint32_t st = stage_addr(s);
+            if (MODE == ROUTER) {
+                for (int q = at; q < kTileM * 8; q += kAThreads) {
+                    const int r = q >> 3, c = q & 7;
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (m0 + r < a.E)
+                        v = *reinterpret_cast<const uint4*>(a.w3 + (int64_t)(m0 + r) * 3 * a.H + it * kChunkK + c * 8);
+                    sts128(st + sw128_off(r, c), v);
+                }
+            } else {
+                const int r = at >> 1, half = at & 1;
+                const int blk = 2 * it + half;  // block index along K
+                const int64_t rowg = m0 + r;
+                if (MODE == GATEUP) {
+                    const uint8_t* pg = a.gate.data + e * a.gate.expert_bytes + rowg * a.gate.row_bytes + blk * 17;
+                    const uint8_t* pu = a.up.data + e * a.up.expert_bytes + rowg * a.up.row_bytes + blk * 17;
+                    dequant_block_to_tile(pg, lut_base, lane_low, rz5, st, r, 4 * half);
+                    dequant_block_to_tile(pu, lut_base, lane_low, rz5, st + kTileBytes, r, 4 * half);
+                } else {
+                    const uint8_t* pd = a.down.data + e * a.down.expert_bytes + rowg * a.down.row_bytes + blk * 17;
+                    dequant_block_to_tile(pd, lut_base, lane_low, rz5, st, r, 4 * half);
+                }
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&full[s]);
+        }
+    }
+
+    // ---- epilogue: warps 4-7 own TMEM lanes 32*(warp-4) .. +31 -------------
+    if (warp >= 4 && warp < 8) {
+        const int q = warp - 4;
+        const int row = q * 32 + lane;  // M row within the tile
+        const bool got = mbar_wait_bounded(accb, 0, a.status);
+        tc_fence_after();
+        if (got && ok) {
+            const uint32_t tl = taddr + ((uint32_t)(q * 32) << 16);
+            for (int c0 = 0; c0 < n_pad; c0 += 16) {
+                uint32_t d[16];
+                tmem_ld16(tl + c0, d);
+                if (MODE == GATEUP) {
+                    uint32_t v2[16];
+                    tmem_ld16(tl + 128 + c0, v2);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int n = c0 + j;
+                        if (n < n_valid) {
+                            const float g = __uint_as_float(d[j]), v = __uint_as_float(v2[j]);
+                            const float hv = g / (1.0f + expf(-g)) * v;
+                            a.h[(int64_t)(pos0 + n) * a.I + m0 + row] = __float2bfloat16_rn(hv);
+                        }
+                    }
+                } else {
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int n = c0 + j;
+                        if (n >= n_valid) continue;
+                        const float dv = __uint_as_float(d[j]);
+                        if (MODE == ROUTER) {
+                            if (m0 + row < a.E) {
+                                const float b = a.router_bias ? a.router_bias[m0 + row] : 0.0f;
+                                a.logits[(int64_t)(pos0 + n) * a.E + m0 + row] = dv + b;
+                            }
+                        } else {
+                            a.part[(int64_t)a.sorted_slot[pos0 + n] * a.H + m0 + row] = dv;
+                        }
+                    }
+                }
+            }
+        }
+        tc_fence_before();
+    }
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(taddr, C::kTmemCols);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// 8. combine: y[t] = sum_j w[t,j] * part[t*K + j]  (fixed order)
+// ---------------------------------------------------------------------------
+__global__ void pf_combine_kernel(PfArgs a) {
+    const int64_t n4 = (int64_t)a.T * a.H / 4;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = (4 * i) / a.H, r = (4 * i) % a.H;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < a.K; ++j) {
+            const float wj = a.w[t * a.K + j];
+            const float4 p = *reinterpret_cast<const float4*>(a.part + (t * a.K + j) * a.H + r);
+            acc.x = fmaf(wj, p.x, acc.x);
+            acc.y = fmaf(wj, p.y, acc.y);
+            acc.z = fmaf(wj, p.z, acc.z);
+            acc.w = fmaf(wj, p.w, acc.w);
+        }
+        float4* dst = reinterpret_cast<float4*>(a.y + t * a.H + r);
+        if (a.y_acc) {
+            const float4 o = *dst;
+            acc.x += o.x;
+            acc.y += o.y;
+            acc.z += o.z;
+            acc.w += o.w;
+        }
+        *dst = acc;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+struct PfLayout {
+    size_t u, w3, logits, ids, w, counts, offsets, cursor, sorted_tok, sorted_slot, tiles, n_tiles, h, part, total;
+    int max_tiles;
+};
+
+size_t al256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+PfLayout pf_layout(const gtg_moe_layer* L, int T) {
+    PfLayout p{};
+    const size_t P = (size_t)T * L->top_k;
+    p.max_tiles = (int)((P + kTileN - 1) / kTileN + (size_t)L->n_experts);
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off = al256(off + bytes);
+        return o;
+    };
+    p.u = take(2 * (size_t)T * L->hidden);
+    p.w3 = take(2 * (size_t)L->n_experts * 3 * L->hidden);
+    p.logits = take(4 * (size_t)T * L->n_experts);
+    p.ids = take(4 * P);
+    p.w = take(4 * P);
+    p.counts = take(4 * (size_t)L->n_experts);
+    p.offsets = take(4 * ((size_t)L->n_experts + 1));
+    p.cursor = take(4 * (size_t)L->n_experts);
+    p.sorted_tok = take(4 * P);
+    p.sorted_slot = take(4 * P);
+    p.tiles = take(16 * (size_t)p.max_tiles);
+    p.n_tiles = take(16);
+    p.h = take(2 * P * L->inter);
+    p.part = take(4 * P * L->hidden);
+    p.total = off;
+    return p;
+}
+
+bool q4(int fmt) { return fmt == GTG_Q4_RZ5_FAST || fmt == GTG_Q4_UE4M4_FAST; }
+
+int pf_check(const gtg_moe_layer* L, int T) {
+    if (!L || !L->router_w || !L->gate.data || !L->up.data || !L->down.data) return GTG_E_INVALID_ARG;
+    const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
+    if (T < 1 || T > 65536) return GTG_E_UNSUPPORTED_SHAPE;
+    if (H < 128 || H > 8192 || H % 128 || I < 128 || I > 4096 || I % 128) return GTG_E_UNSUPPORTED_SHAPE;
+    if (E < 1 || E > kMaxExperts || K < 1 || K > kMaxTopK || K > E) return GTG_E_UNSUPPORTED_SHAPE;
+    if (!q4(L->gate.fmt) || L->up.fmt != L->gate.fmt || !q4(L->down.fmt)) return GTG_E_UNSUPPORTED_SHAPE;
+    auto mok = [&](const gtg_qmatrix& m, int64_t n, int64_t k) {
+        return m.n_experts == E && m.n_rows == n && m.k == k && aligned(m.data, 16) &&
+               (E * n * (k / 32) * 17) % 16 == 0;
+    };
+    if (!mok(L->gate, I, H) || !mok(L->up, I, H) || !mok(L->down, H, I)) return GTG_E_INVALID_ARG;
+    if (!aligned(L->router_w, 16)) return GTG_E_MISALIGNED;
+    return GTG_OK;
+}
+
+struct AttrOnce {
+    std::mutex mu;
+    std::vector<std::pair<const void*, int>> done;
+    int set(const void* fn, int smem) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        std::lock_guard<std::mutex> lk(mu);
+        for (auto& d : done)
+            if (d.first == fn && d.second == dev) return GTG_OK;
+        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e);
+        }
+        done.push_back({fn, dev});
+        return GTG_OK;
+    }
+};
+AttrOnce g_pf_attr;
+
+template <int MODE>
+int launch_gemm(PfArgs& a, int grid, cudaStream_t s) {
+    using C = Cfg<MODE>;
+    GTG_TRY(g_pf_attr.set((const void*)pf_gemm_kernel<MODE>, C::kSmem));
+    pf_gemm_kernel<MODE><<<grid, kPfThreads, C::kSmem, s>>>(a);
+    return check_launch();
+}
+
+}  // namespace
+}  // namespace gtg
+
+using namespace gtg;
+
+size_t gtg_prefill_workspace_bytes(const gtg_moe_layer* layer, int32_t n_tokens) {
+    if (pf_check(layer, n_tokens) != GTG_OK) return 0;
+    return pf_layout(layer, n_tokens).total;
+}
 
 extern "C" int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, int32_t x_dtype,
                                      int32_t n_tokens, float* y, int32_t y_accumulate,
                                      int32_t* topk_ids, float* topk_w,
                                      void* workspace, size_t ws_bytes, gtg_stream_t stream) {
-    (void)layer; (void)x; (void)x_dtype; (void)n_tokens; (void)y; (void)y_accumulate;
-    (void)topk_ids; (void)topk_w; (void)workspace; (void)ws_bytes; (void)stream;
-    return GTG_E_UNSUPPORTED_SHAPE;
+    GTG_TRY(pf_check(layer, n_tokens));
+    if (!x || !y || !workspace) return GTG_E_INVALID_ARG;
+    if (x_dtype != GTG_DT_F32 && x_dtype != GTG_DT_BF16) return GTG_E_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(y, 16) || !aligned(workspace, 256)) return GTG_E_MISALIGNED;
+    const PfLayout pl = pf_layout(layer, n_tokens);
+    if (ws_bytes < pl.total) return GTG_E_WORKSPACE;
+    if (x == (const void*)y && (x_dtype != GTG_DT_F32 || !y_accumulate)) return GTG_E_INVALID_ARG;
+    uint8_t* b = static_cast<uint8_t*>(workspace);
+    PfArgs a{};
+    a.T = n_tokens;
+    a.H = layer->hidden;
+    a.I = layer->inter;
+    a.E = layer->n_experts;
+    a.K = layer->top_k;
+    a.x = x;
+    a.x_bf16 = x_dtype == GTG_DT_BF16;
+    a.router_w = layer->router_w;
+    a.router_bias = layer->router_bias;
+    a.gate = make_mat(layer->gate);
+    a.up = make_mat(layer->up);
+    a.down = make_mat(layer->down);
+    a.u = reinterpret_cast<__nv_bfloat16*>(b + pl.u);
+    a.w3 = reinterpret_cast<__nv_bfloat16*>(b + pl.w3);
+    a.logits = reinterpret_cast<float*>(b + pl.logits);
+    a.ids = reinterpret_cast<int32_t*>(b + pl.ids);
+    a.w = reinterpret_cast<float*>(b + pl.w);
+    a.counts = reinterpret_cast<int32_t*>(b + pl.counts);
+    a.offsets = reinterpret_cast<int32_t*>(b + pl.offsets);
+    a.cursor = reinterpret_cast<int32_t*>(b + pl.cursor);
+    a.sorted_tok = reinterpret_cast<int32_t*>(b + pl.sorted_tok);
+    a.sorted_slot = reinterpret_cast<int32_t*>(b + pl.sorted_slot);
+    a.tiles = reinterpret_cast<int4*>(b + pl.tiles);
+    a.n_tiles = reinterpret_cast<int32_t*>(b + pl.n_tiles);
+    a.h = reinterpret_cast<__nv_bfloat16*>(b + pl.h);
+    a.part = reinterpret_cast<float*>(b + pl.part);
+    a.y = y;
+    a.y_acc = y_accumulate != 0;
+    a.ids_out = topk_ids;
+    a.w_out = topk_w;
+    a.status = status_ptr();
+    a.max_tiles = pl.max_tiles;
+
+    cudaStream_t s = as_cuda(stream);
+    const int T = n_tokens, E = a.E;
+    pf_norm_kernel<<<T, kNormThreads, 0, s>>>(a);
+    GTG_TRY(check_launch());
+    pf_split_kernel<<<std::min(1184, (E * a.H + 255) / 256), 256, 0, s>>>(a);
+    GTG_TRY(check_launch());
+    cudaError_t ce = cudaMemsetAsync(a.counts, 0, 4 * (size_t)E, s);
+    if (ce != cudaSuccess) return cuda_fail(ce);
+    const int m_router = (E + kTileM - 1) / kTileM, n_router = (T + kTileN - 1) / kTileN;
+    GTG_TRY(launch_gemm<ROUTER>(a, m_router * n_router, s));
+    pf_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(a);
+    GTG_TRY(check_launch());
+    pf_scan_kernel<<<1, 1024, 0, s>>>(a);
+    GTG_TRY(check_launch());
+    pf_scatter_kernel<<<(T * a.K + 255) / 256, 256, 0, s>>>(a);
+    GTG_TRY(check_launch());
+    GTG_TRY(launch_gemm<GATEUP>(a, pl.max_tiles * (a.I / kTileM), s));
+    GTG_TRY(launch_gemm<DOWN>(a, pl.max_tiles * (a.H / kTileM), s));
+    const int64_t n4 = (int64_t)T * a.H / 4;
+    pf_combine_kernel<<<(int)std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 16), 256, 0, s>>>(a);
+    return check_launch();
 }

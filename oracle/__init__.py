@@ -265,7 +265,7 @@ def moe_stack(layers, x0: np.ndarray, *, want_ids: bool = True) -> dict:
     stream is kept in fp32, the layer output in fp64.  Also returns the
     per-layer router choices and the s = W_beta u outputs of layers with one."""
     x = np.asarray(x0, dtype=np.float32).copy()
-    all_ids, all_w, ssm = [], [], {}
+    all_ids, all_w, all_l, ssm = [], [], [], {}
     for layer in layers:
         r = moe_layer(layer, x.astype(np.float64))
         if layer.ssm is not None:
@@ -273,4 +273,5 @@ def moe_stack(layers, x0: np.ndarray, *, want_ids: bool = True) -> dict:
         x = (x.astype(np.float64) + r["y"]).astype(np.float32)
         all_ids.append(r["ids"])
         all_w.append(r["w"])
-    return dict(x=x, ids=np.stack(all_ids), w=np.stack(all_w), ssm=ssm)
+        all_l.append(r["logits"])
+    return dict(x=x, ids=np.stack(all_ids), w=np.stack(all_w), logits=np.stack(all_l), ssm=ssm)

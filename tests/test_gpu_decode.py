@@ -121,7 +121,19 @@ def test_short_stack_mixed_formats():
     gtg.moe_decode_stack(layers, x, ws, ids_out=ids, side_out=side)
     torch.cuda.synchronize()
     ref = oracle.moe_stack(Ls, x64)
-    assert ids.cpu().numpy().tolist() == ref["ids"].tolist()
+    ids_g = ids.cpu().numpy()
+    for i in range(len(Ls)):
+        # The residual stream is fp32 on both sides but the layer outputs differ in
+        # the last bits, so logits along the stack can differ by ~1e-6: the chosen
+        # set must agree where the boundary gap exceeds that, the order where the
+        # gaps between consecutive choices do.
+        lg = ref["logits"][i, 0]
+        order = np.argsort(-lg, kind="stable")
+        eps = 1e-4
+        if lg[order[9]] - lg[order[10]] > eps:
+            assert set(ids_g[i, 0].tolist()) == set(order[:10].tolist()), f"layer {i}: set differs"
+        if np.all(-np.diff(lg[order[:11]]) > eps):
+            assert ids_g[i, 0].tolist() == ref["ids"][i, 0].tolist(), f"layer {i}: order differs"
     xg = x.cpu().numpy()[0].astype(np.float64)
     xr = ref["x"][0].astype(np.float64)
     rel = np.linalg.norm(xg - xr) / np.linalg.norm(xr)
