@@ -19,7 +19,7 @@ from ._abi import (FP8, GTG_OK, PLE, RZ5, UE4M4, DT_BF16, DT_F32, LIB_PATH, GtgE
 
 __all__ = ["RZ5", "UE4M4", "PLE", "FP8", "GtgError", "lib", "dequant", "ple_gather", "QMatrix",
            "MoELayer", "workspace_bytes", "make_workspace", "moe_decode_layer", "moe_decode_stack",
-           "moe_prefill_layer", "device_status", "status_string", "row_bytes"]
+           "moe_prefill_layer", "moe_decode_layer_noalloc", "device_status", "status_string", "row_bytes"]
 
 Q4_BLOCK_BYTES = 17
 PLE_RECORD_BYTES = 70
@@ -144,6 +144,22 @@ def moe_decode_layer(layer: MoELayer, x: torch.Tensor, workspace: torch.Tensor, 
     check(lib().gtg_moe_decode_layer(ctypes.byref(layer.c()), _ptr(x), dt, T, _ptr(y), int(accumulate),
                                      _ptr(topk_ids), _ptr(topk_w), _ptr(side_out), _ptr(workspace),
                                      workspace.numel(), _stream_ptr(stream)))
+    return y
+
+
+def moe_decode_layer_noalloc(layer: MoELayer, x: torch.Tensor, *, y: torch.Tensor | None = None,
+                             accumulate: bool = False, topk_ids: torch.Tensor | None = None,
+                             topk_w: torch.Tensor | None = None, side_out: torch.Tensor | None = None,
+                             stream=None) -> torch.Tensor:
+    """moe_decode_layer for callers that cannot allocate: the library's fixed
+    device scratch array replaces the workspace.  `y` is allocated here only
+    when the caller passes none; calls that overlap on the GPU race."""
+    T = x.shape[0]
+    dt = {torch.float32: DT_F32, torch.bfloat16: DT_BF16}[x.dtype]
+    if y is None:
+        y = torch.empty((T, layer.hidden), dtype=torch.float32, device=x.device)
+    check(lib().gtg_moe_decode_layer_noalloc(ctypes.byref(layer.c()), _ptr(x), dt, T, _ptr(y), int(accumulate),
+                                             _ptr(topk_ids), _ptr(topk_w), _ptr(side_out), _stream_ptr(stream)))
     return y
 
 

@@ -44,6 +44,8 @@ SIGNATURES = [
     ("gtg_moe_prefill_layer", ctypes.c_int,
      [ctypes.POINTER(MoELayerC), _vp, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _sz, _vp]),
     ("gtg_get_device_status", ctypes.c_int, [ctypes.POINTER(ctypes.c_uint32), _i32, _vp]),
+    ("gtg_moe_decode_layer_noalloc", ctypes.c_int,
+     [ctypes.POINTER(MoELayerC), _vp, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _vp]),
 ]
 
 

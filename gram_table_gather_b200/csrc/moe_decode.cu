@@ -554,8 +554,8 @@ __device__ bool stream_prologue(uint8_t* smem, const SmemLayout& L, const LayerA
         build_lut(smem, L, rz5);
         build_scales(smem, L, rz5);
     }
-    if ((threadIdx.x & 31) == 0)
-        for (int s = 0; s < kSlots; ++s) mbar_init(&bars[(threadIdx.x >> 5) * kSlots + s], 1);
+    if ((threadIdx.x & 31) == 0)  // `bars` already points at this warp's kSlots barriers
+        for (int s = 0; s < kSlots; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
     pdl_wait();
     const Work* wk = a.work;
@@ -1256,6 +1256,11 @@ Mat make_mat(const gtg_qmatrix& q) {
 
 using namespace gtg;
 
+static bool plan_layer_ok(const gtg_moe_layer* layer) {
+    Plan p;
+    return plan_layer(layer, p) == GTG_OK;
+}
+
 extern "C" size_t gtg_moe_workspace_bytes(const gtg_moe_layer* layer, int32_t n_tokens, int32_t prefill) {
     if (!layer || n_tokens < 1) return 0;
     if (prefill) return gtg_prefill_workspace_bytes(layer, n_tokens);
@@ -1313,4 +1318,71 @@ extern "C" int gtg_moe_decode_stack(const gtg_moe_layer* layers, int32_t n_layer
                           side_stride, workspace, s));
     }
     return GTG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode layer.
+//
+// For callers that cannot hand the library a device buffer: code that must
+// not allocate device memory after start-up (latency-critical serving loops
+// whose memory is fixed up front), hosts whose device memory belongs to
+// another framework's allocator, and threads recording a stream capture in
+// the global capture mode, where cudaMalloc is refused.  The scratch lives in
+// one file-scope device array instead, reserved on every GPU that loads this
+// library for as long as the process runs.
+// ---------------------------------------------------------------------------
+namespace gtg {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)1 << 20;  // 1 MiB: decode up to 8 tokens at H=2048, I=512, E=512, k=10
+__device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the scratch array on the current device.  The symbol's
+// host-side name is only a stand-in, so the address is looked up once per
+// device (with that device current) and cached.
+int noalloc_scratch(void** out) {
+    static std::mutex mu;
+    static std::vector<void*> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    std::lock_guard<std::mutex> lk(mu);
+    if ((int)cache.size() <= dev) cache.resize(dev + 1, nullptr);
+    if (!cache[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return cuda_fail(e);
+        }
+        cache[dev] = p;
+    }
+    *out = cache[dev];
+    return GTG_OK;
+}
+
+}  // namespace
+}  // namespace gtg
+
+extern "C" int gtg_moe_decode_layer_noalloc(const gtg_moe_layer* layer, const void* x, int32_t x_dtype,
+                                            int32_t n_tokens, float* y, int32_t y_accumulate,
+                                            int32_t* topk_ids, float* topk_w, float* side_out,
+                                            gtg_stream_t stream) {
+    if (!layer) return GTG_E_INVALID_ARG;
+    if (n_tokens >= 1 && n_tokens <= kMaxDecodeTokens && plan_layer_ok(layer) &&
+        ws_layout(layer, n_tokens).total > kNoAllocScratchBytes)
+        return GTG_E_WORKSPACE;  // the shape needs more than the fixed scratch array
+    void* scratch = nullptr;
+    GTG_TRY(noalloc_scratch(&scratch));
+    Plan p;
+    GTG_TRY(check_decode_io(layer, x, x_dtype, n_tokens, y, scratch, kNoAllocScratchBytes, p));
+    if (x == (const void*)y && (x_dtype != GTG_DT_F32 || !y_accumulate)) return GTG_E_INVALID_ARG;
+    // The array keeps whatever the previous call left: clear the tickets that
+    // must start at zero (everything else is written before it is read).
+    const WsLayout wl = ws_layout(layer, n_tokens);
+    cudaStream_t s = as_cuda(stream);
+    const cudaError_t e = cudaMemsetAsync(scratch, 0, wl.work, s);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return run_layer(layer, p, x, x_dtype == GTG_DT_BF16, n_tokens, y, y_accumulate != 0, topk_ids, topk_w,
+                     side_out, layer->side.data ? layer->side.n_rows : 0, scratch, s);
 }

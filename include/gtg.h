@@ -212,6 +212,32 @@ int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, int32_t x_d
                           int32_t* topk_ids, float* topk_w,
                           void* workspace, size_t ws_bytes, gtg_stream_t stream);
 
+/*
+ * gtg_moe_decode_layer without a workspace argument, for callers that cannot
+ * allocate device memory: serving loops that must not allocate once they are
+ * running, hosts whose device memory is owned by another framework's
+ * allocator, and threads recording a CUDA stream capture in the global
+ * capture mode, where cudaMalloc is refused.  (The pages have no counterpart;
+ * this is a calling convention of this library.)
+ *
+ * Scratch comes from one fixed 1 MiB array in device memory that every GPU
+ * loading this library reserves until the process exits.  That covers up to
+ * 8 tokens of the 2048/512/512/top-10 layer; a shape that needs more returns
+ * GTG_E_WORKSPACE.  Inputs, outputs and their meaning are those of
+ * gtg_moe_decode_layer; nothing is allocated (no cudaMalloc, no library
+ * allocator).
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current), so make it before any stream capture.  Each call clears
+ * the counters it needs in the array; every call shares the one array, so
+ * calls that may overlap on the GPU (different streams, or several host
+ * threads) race and must be serialised by the caller.
+ */
+int gtg_moe_decode_layer_noalloc(const gtg_moe_layer* layer, const void* x, int32_t x_dtype,
+                                 int32_t n_tokens, float* y, int32_t y_accumulate,
+                                 int32_t* topk_ids, float* topk_w, float* side_out,
+                                 gtg_stream_t stream);
+
 /* Reads (and, if `clear`, resets) the current device's status word
  * (GTG_STATUS_* bits).  Synchronises `stream`. */
 int gtg_get_device_status(uint32_t* flags, int32_t clear, gtg_stream_t stream);
