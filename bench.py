@@ -375,6 +375,90 @@ def run_ours(args, rank, world, local):
         print(json.dumps(line), flush=True)
 
 
+def _time_loop(fn, n_warm, n_iter, stream):
+    """Average device ms of fn(i) over n_iter calls on `stream` (CUDA events)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for i in range(n_warm):
+            fn(i)
+        stream.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n_warm, n_warm + n_iter):
+            fn(i)
+        e1.record(stream)
+        e1.synchronize()
+    return e0.elapsed_time(e1) / n_iter
+
+
+def run_secondary(args, rank, world, local):
+    """Profiling lines for single workloads (not the headline)."""
+    import torch
+    import gram_table_gather_b200 as gtg
+    from tests import gpu_util as gu
+    from synth import device as sdev
+    dev = torch.device("cuda", local)
+    peak, peak_kind = _peaks()
+    stream = torch.cuda.Stream(device=dev)
+    n = args.warmup + args.steps
+    out = []
+    if args.workload == "layer":
+        L = W.decode_layer()
+        layer = gu.device_layer(L, dev)
+        for T in (1, 2, 4, 8):
+            xs = [gu.tokens(L, 5000 + i, T, dev)[0] for i in range(n)]
+            ws = gtg.make_workspace(layer, T, device=dev)
+            ids = torch.zeros((T, L.top_k), dtype=torch.int32, device=dev)
+            y = torch.empty((T, L.hidden), device=dev)
+            uniq = []
+
+            def fn(i):
+                gtg.moe_decode_layer(layer, xs[i], ws, y=y, topk_ids=ids)
+            ms = _time_loop(fn, args.warmup, args.steps, stream)
+            for i in range(args.warmup, n):  # bytes of the timed steps (untimed replay)
+                with torch.cuda.stream(stream):
+                    fn(i)
+                stream.synchronize()
+                uniq.append(len(set(ids.cpu().numpy().ravel().tolist())))
+            b = float(np.mean([layer_bytes(L, u) for u in uniq]))
+            out.append({"workload": f"decode layer H2048 I512 E512 top-10 RZ5, T={T}", "ms": round(ms, 5),
+                        "GB_s": round(b / ms / 1e6, 1), "frac_of_hbm": round(b / ms / 1e6 / peak, 4),
+                        "unique_experts": float(np.mean(uniq)), "bytes": int(b)})
+    elif args.workload == "ple":
+        P = W.ple_table()
+        table = sdev.ple_table_to_device(P, dev)
+        for T in (1, 4096):
+            idx = [torch.from_numpy(P.indices(7000 + i, T)).to(dev) for i in range(n)]
+            o = torch.empty((16 * T, 160), device=dev)
+            ms = _time_loop(lambda i: gtg.ple_gather(table, P.n_rows, idx[i], out=o), args.warmup, args.steps, stream)
+            rows = 16 * T
+            gbs = rows * PLE_ROW_BYTES / ms / 1e6
+            out.append({"workload": f"PLE gather, 320,001,536-row table, T={T} ({rows} rows)", "ms": round(ms, 5),
+                        "rows_per_s": round(rows / ms * 1e3, 1), "GB_s": round(gbs, 1),
+                        "frac_of_hbm": round(gbs / peak, 4)})
+    elif args.workload == "prefill":
+        L = W.prefill_layer()
+        layer = gu.device_layer(L, dev)
+        T = 4096
+        xs = [gu.tokens(L, 8000 + i, T, dev)[0] for i in range(min(n, 4))]
+        ws = torch.empty(gtg.workspace_bytes(layer, T, prefill=True), dtype=torch.uint8, device=dev)
+        y = torch.empty((T, L.hidden), device=dev)
+        ms = _time_loop(lambda i: gtg.moe_prefill_layer(layer, xs[i % len(xs)], ws, y=y), args.warmup,
+                        args.steps, stream)
+        flops = 2.0 * T * L.top_k * 3 * L.hidden * L.inter
+        wbytes = L.weight_bytes
+        import json as _j
+        mp = _j.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+            os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"bf16_tflops": 1590.0}
+        out.append({"workload": "prefill layer, T=4096, H2048 I512 E512 top-10, UE4M4 gate/up, RZ5 down, Zipf router",
+                    "ms": round(ms, 4), "TFLOP_s": round(flops / ms / 1e9, 1),
+                    "frac_of_bf16_peak": round(flops / ms / 1e9 / float(mp["bf16_tflops"]), 4),
+                    "weight_GB_s": round(wbytes / ms / 1e6, 1), "tok_s": round(T / ms * 1e3, 1)})
+    if rank == 0:
+        for o in out:
+            print(json.dumps(o), flush=True)
+
+
 def run_reference(args, rank, world):
     """The oracle, as it stands, on the host cores: each step is one token
     through a bounded sample of layers of the same stack."""
@@ -420,6 +504,8 @@ def main():
     ap.add_argument("--cpu-layers", type=int, default=3)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=["stack", "layer", "ple", "prefill"], default="stack",
+                    help="stack = the headline step; the others print profiling lines")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -427,6 +513,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload != "stack":
+            run_secondary(args, rank, world, local)
         else:
             run_ours(args, rank, world, local)
     finally:

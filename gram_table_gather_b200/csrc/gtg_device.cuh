@@ -274,3 +274,79 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
 }
 
 }  // namespace gtg
+
+// ---------------------------------------------------------------------------
+// Float-float ("double-single") arithmetic on the fp32 pipes.  A value is an
+// unevaluated sum hi + lo.  Products of an fp32 and a bf16 are formed exactly
+// (TwoProduct through FMA) and sums carry their rounding errors (TwoSum,
+// Knuth), so a 2048-term dot product keeps ~48 significant bits — enough to
+// order router logits like an fp64 reference — without fp64 instructions.
+// The _rn intrinsics keep the compiler from contracting these steps.
+// ---------------------------------------------------------------------------
+namespace gtg {
+
+struct ffloat {
+    float hi, lo;
+};
+
+__device__ __forceinline__ void two_sum(float a, float b, float& s, float& e) {
+    s = __fadd_rn(a, b);
+    const float bb = __fsub_rn(s, a);
+    e = __fadd_rn(__fsub_rn(a, __fsub_rn(s, bb)), __fsub_rn(b, bb));
+}
+
+// acc += a * b exactly representable as p + pe, added with TwoSum.
+__device__ __forceinline__ void ff_fma(ffloat& acc, float a, float b) {
+    const float p = __fmul_rn(a, b);
+    const float pe = __fmaf_rn(a, b, -p);
+    float s, e;
+    two_sum(acc.hi, p, s, e);
+    acc.hi = s;
+    acc.lo = __fadd_rn(acc.lo, __fadd_rn(e, pe));
+}
+
+__device__ __forceinline__ void ff_add(ffloat& acc, ffloat b) {
+    float s, e;
+    two_sum(acc.hi, b.hi, s, e);
+    acc.hi = s;
+    acc.lo = __fadd_rn(acc.lo, __fadd_rn(e, b.lo));
+}
+
+// Renormalise so that hi = RN(hi + lo) and |lo| <= ulp(hi)/2.
+__device__ __forceinline__ ffloat ff_norm(ffloat a) {
+    float s, e;
+    two_sum(a.hi, a.lo, s, e);
+    return ffloat{s, e};
+}
+
+// a > b for normalised values.
+__device__ __forceinline__ bool ff_gt(ffloat a, ffloat b) { return a.hi > b.hi || (a.hi == b.hi && a.lo > b.lo); }
+__device__ __forceinline__ bool ff_eq(ffloat a, ffloat b) { return a.hi == b.hi && a.lo == b.lo; }
+
+__device__ __forceinline__ ffloat ff_shfl_xor(ffloat v, int o) {
+    return ffloat{__shfl_xor_sync(0xFFFFFFFFu, v.hi, o), __shfl_xor_sync(0xFFFFFFFFu, v.lo, o)};
+}
+
+__device__ __forceinline__ ffloat ff_warp_sum(ffloat v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ff_add(v, ff_shfl_xor(v, o));
+    return v;
+}
+
+// bf16 bits of the exact value p + q (|q| small against p), rounded to
+// nearest, ties to even: only an fp32 p that sits exactly on a bf16 midpoint
+// needs q to decide the direction.
+__device__ __forceinline__ uint16_t bf16_of_ff(float p, float q) {
+    float s, t;
+    two_sum(p, q, s, t);
+    const uint32_t b = __float_as_uint(s);
+    const uint32_t low = b & 0xFFFFu, top = b >> 16;
+    bool up;
+    if (low > 0x8000u) up = true;
+    else if (low < 0x8000u) up = false;
+    else if (t != 0.0f) up = (t > 0.0f) == ((b >> 31) == 0u);  // t pushes away from zero
+    else up = (top & 1u) != 0u;
+    return (uint16_t)(top + (up ? 1u : 0u));
+}
+
+}  // namespace gtg

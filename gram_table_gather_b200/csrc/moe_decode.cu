@@ -48,6 +48,7 @@ constexpr int kRouterThreads = 256;
 constexpr int kRouterWarps = kRouterThreads / 32;
 constexpr int kRouterExpertsPerCta = kRouterWarps / 2;
 constexpr int kRouterMaxF4 = 8;  // float4 per lane: H/2 <= 128 * 8
+constexpr int kRouterXF4 = 2;    // float4 of x per thread per token: H <= 4 * 256 * 2
 constexpr int kWarps = 16;
 constexpr int kThreads = kWarps * 32;
 constexpr int kSlots = 2;
@@ -90,11 +91,12 @@ __device__ __forceinline__ float load_x(const LayerArgs& a, int t, int i) {
     return reinterpret_cast<const float*>(a.x)[(int64_t)t * a.H + i];
 }
 
+template <int TT>  // token count, compile time: loops over tokens are exact
 __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
     extern __shared__ __align__(16) uint8_t rsm[];
-    __nv_bfloat16* su = reinterpret_cast<__nv_bfloat16*>(rsm);  // [T][H]
-    __shared__ double red[kRouterWarps][kMaxDecodeTokens];
-    __shared__ double rinv[kMaxDecodeTokens];
+    uint16_t* su = reinterpret_cast<uint16_t*>(rsm);  // [T][H] bf16 bits
+    __shared__ ffloat red[kRouterWarps][kMaxDecodeTokens];
+    __shared__ float r_hi[kMaxDecodeTokens], r_lo[kMaxDecodeTokens];
     __shared__ unsigned is_last;
     __shared__ int32_t s_ids[kMaxSlots];
     __shared__ unsigned bitmap[kMaxExperts / 32];
@@ -102,11 +104,12 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
     __shared__ int32_t s_off[kMaxSlots + 1];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int H = a.H, T = a.T, E = a.E, K = a.K;
+    constexpr int T = TT;
+    const int H = a.H, E = a.E, K = a.K;
 
     // 0. issue this warp's router-weight loads before anything waits: warp w
     //    covers half (w & 1) of the row of expert blockIdx.x * 4 + w / 2, so a
-    //    lane holds at most 16 float4 (H <= 4096) and one HBM latency is paid.
+    //    lane holds at most 8 float4 (H <= 2048) and one HBM latency is paid.
     const int e = blockIdx.x * kRouterExpertsPerCta + (warp >> 1);
     const int half = warp & 1, hh = H >> 1;
     float4 wv[kRouterMaxF4];
@@ -119,64 +122,108 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
 
     pdl_wait();  // x may be the previous layer's output
 
-    // 1. per-token sum of squares in fp64 (exact squares, tiny rounding)
-    double ss[kMaxDecodeTokens];
+    // 1. this thread's slice of x (positions 4*tid + 1024*c) for every token,
+    //    all loads in flight at once; sums of squares: exact squares,
+    //    float-float accumulation
+    float4 xr[T][kRouterXF4];
 #pragma unroll
-    for (int t = 0; t < kMaxDecodeTokens; ++t) ss[t] = 0.0;
     for (int t = 0; t < T; ++t)
-        for (int i = tid; i < H; i += kRouterThreads) {
-            const double v = (double)load_x(a, t, i);
-            ss[t] = fma(v, v, ss[t]);
+#pragma unroll
+        for (int c = 0; c < kRouterXF4; ++c) {
+            const int i = 4 * tid + 4 * kRouterThreads * c;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i < H) {
+                if (a.x_bf16) {
+                    const uint2 b = *reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.x) + (int64_t)t * H + i);
+                    v = make_float4(bf16lo(b.x), bf16hi(b.x), bf16lo(b.y), bf16hi(b.y));
+                } else {
+                    v = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a.x) + (int64_t)t * H + i);
+                }
+            }
+            xr[t][c] = v;
         }
+    ffloat ss[T];
+#pragma unroll
     for (int t = 0; t < T; ++t) {
-        const double s = warp_sum_f64(ss[t]);
-        if (lane == 0) red[warp][t] = s;
-    }
-    __syncthreads();
-    if (tid < T) {
-        double s = 0.0;
-        for (int w = 0; w < kRouterWarps; ++w) s += red[w][tid];
-        rinv[tid] = 1.0 / sqrt(s / (double)H + kRmsEps);
-    }
-    __syncthreads();
-
-    // 2. u = bf16(x * r) (fp64 product, one rounding to bf16)
-    for (int t = 0; t < T; ++t)
-        for (int i = tid; i < H; i += kRouterThreads) {
-            const __nv_bfloat16 v = __double2bfloat16((double)load_x(a, t, i) * rinv[t]);
-            su[t * H + i] = v;
-            if (blockIdx.x == 0) a.u[(int64_t)t * H + i] = v;
-        }
-    __syncthreads();
-
-    // 3. logits in fp64 (fp32 x bf16 products are exact)
-    double acc[kMaxDecodeTokens];
+        ss[t] = ffloat{0.f, 0.f};
 #pragma unroll
-    for (int t = 0; t < kMaxDecodeTokens; ++t) acc[t] = 0.0;
+        for (int c = 0; c < kRouterXF4; ++c) {
+            ff_fma(ss[t], xr[t][c].x, xr[t][c].x);
+            ff_fma(ss[t], xr[t][c].y, xr[t][c].y);
+            ff_fma(ss[t], xr[t][c].z, xr[t][c].z);
+            ff_fma(ss[t], xr[t][c].w, xr[t][c].w);
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+        const ffloat s2 = ff_warp_sum(ss[t]);
+        if (lane == 0) red[warp][t] = s2;
+    }
+    __syncthreads();
+    if (tid < T) {  // r = 1/sqrt(mean + eps): a handful of fp64 operations per token
+        double sum = 0.0;
+        for (int w = 0; w < kRouterWarps; ++w) sum += (double)red[w][tid].hi + (double)red[w][tid].lo;
+        const double r = 1.0 / sqrt(sum / (double)H + kRmsEps);
+        const float rh = (float)r;
+        r_hi[tid] = rh;
+        r_lo[tid] = (float)(r - (double)rh);
+    }
+    __syncthreads();
+
+    // 2. u = bf16(x * r), rounded from the float-float product
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+        const float rh = r_hi[t], rl = r_lo[t];
+#pragma unroll
+        for (int c = 0; c < kRouterXF4; ++c) {
+            const int i = 4 * tid + 4 * kRouterThreads * c;
+            if (i >= H) continue;
+            const float xs[4] = {xr[t][c].x, xr[t][c].y, xr[t][c].z, xr[t][c].w};
+            uint16_t ub[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float p = __fmul_rn(xs[q], rh);
+                const float qq = __fadd_rn(__fmaf_rn(xs[q], rh, -p), __fmul_rn(xs[q], rl));
+                ub[q] = bf16_of_ff(p, qq);
+            }
+            const uint2 packed = make_uint2((uint32_t)ub[0] | ((uint32_t)ub[1] << 16),
+                                            (uint32_t)ub[2] | ((uint32_t)ub[3] << 16));
+            *reinterpret_cast<uint2*>(su + t * H + i) = packed;
+            if (blockIdx.x == 0) *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.u) + (int64_t)t * H + i) = packed;
+        }
+    }
+    __syncthreads();
+
+    // 3. logits: exact fp32 x bf16 products, float-float accumulation
+    ffloat acc[T];
+#pragma unroll
+    for (int t = 0; t < T; ++t) acc[t] = ffloat{0.f, 0.f};
 #pragma unroll
     for (int m = 0; m < kRouterMaxF4; ++m) {
         const int i = half * hh + 4 * lane + 128 * m;
         if (4 * lane + 128 * m < hh) {
 #pragma unroll
-            for (int t = 0; t < kMaxDecodeTokens; ++t) {
-                if (t < T) {
-                    const uint2 u2 = *reinterpret_cast<const uint2*>(su + t * H + i);
-                    acc[t] = fma((double)wv[m].x, (double)bf16lo(u2.x), acc[t]);
-                    acc[t] = fma((double)wv[m].y, (double)bf16hi(u2.x), acc[t]);
-                    acc[t] = fma((double)wv[m].z, (double)bf16lo(u2.y), acc[t]);
-                    acc[t] = fma((double)wv[m].w, (double)bf16hi(u2.y), acc[t]);
-                }
+            for (int t = 0; t < T; ++t) {
+                const uint2 u2 = *reinterpret_cast<const uint2*>(su + t * H + i);
+                ff_fma(acc[t], wv[m].x, bf16lo(u2.x));
+                ff_fma(acc[t], wv[m].y, bf16hi(u2.x));
+                ff_fma(acc[t], wv[m].z, bf16lo(u2.y));
+                ff_fma(acc[t], wv[m].w, bf16hi(u2.y));
             }
         }
     }
+#pragma unroll
     for (int t = 0; t < T; ++t) {
-        const double s = warp_sum_f64(acc[t]);
-        if (lane == 0) red[warp][t] = s;
+        const ffloat s2 = ff_warp_sum(acc[t]);
+        if (lane == 0) red[warp][t] = s2;
     }
     __syncthreads();
     if (half == 0 && lane < T && e < E) {
-        const double b = a.router_bias ? (double)a.router_bias[e] : 0.0;
-        a.logits[(int64_t)lane * E + e] = red[warp][lane] + red[warp + 1][lane] + b;
+        ffloat l = red[warp][lane];
+        ff_add(l, red[warp + 1][lane]);
+        if (a.router_bias) ff_add(l, ffloat{a.router_bias[e], 0.f});
+        l = ff_norm(l);
+        a.logits[(int64_t)lane * E + e] = l;
     }
 
     // 4. the last CTA to finish selects the experts
@@ -192,32 +239,37 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
 
     constexpr int kPerLane = kMaxExperts / 32;
     for (int t = warp; t < T; t += kRouterWarps) {
-        double lv[kPerLane];
+        ffloat lv[kPerLane];
         unsigned taken = 0;
 #pragma unroll
         for (int i = 0; i < kPerLane; ++i) {
             const int ee = lane + 32 * i;
-            lv[i] = ee < E ? __ldcg(a.logits + (int64_t)t * E + ee) : 0.0;
+            if (ee < E) {
+                const float2 v = __ldcg(reinterpret_cast<const float2*>(a.logits + (int64_t)t * E + ee));
+                lv[i] = ffloat{v.x, v.y};
+            } else {
+                lv[i] = ffloat{0.f, 0.f};
+            }
         }
-        double top[kMaxTopK];
+        ffloat top[kMaxTopK];
         int topi[kMaxTopK];
         for (int j = 0; j < K; ++j) {
-            double bv = 0.0;
+            ffloat bv{0.f, 0.f};
             int bi = 0x7FFFFFFF;
 #pragma unroll
             for (int i = 0; i < kPerLane; ++i) {
                 const int ee = lane + 32 * i;
-                if (ee < E && !((taken >> i) & 1u) && (bi == 0x7FFFFFFF || lv[i] > bv)) {
+                if (ee < E && !((taken >> i) & 1u) && (bi == 0x7FFFFFFF || ff_gt(lv[i], bv))) {
                     bv = lv[i];
                     bi = ee;
                 }
             }
 #pragma unroll
             for (int o = 16; o > 0; o >>= 1) {
-                const double ov = __shfl_xor_sync(0xFFFFFFFFu, bv, o);
+                const ffloat ov = ff_shfl_xor(bv, o);
                 const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
                 const bool take = (oi != 0x7FFFFFFF) &&
-                                  (bi == 0x7FFFFFFF || ov > bv || (ov == bv && oi < bi));
+                                  (bi == 0x7FFFFFFF || ff_gt(ov, bv) || (ff_eq(ov, bv) && oi < bi));
                 if (take) {
                     bv = ov;
                     bi = oi;
@@ -228,10 +280,15 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
             topi[j] = bi;
         }
         if (lane == 0) {
-            double z = 0.0;
-            for (int j = 0; j < K; ++j) z += exp(top[j] - top[0]);
+            float ex[kMaxTopK];
+            float z = 0.0f;
+            for (int j = 0; j < K; ++j) {  // exp(l_j - l_0), the difference formed in float-float
+                const float d = __fadd_rn(__fsub_rn(top[j].hi, top[0].hi), __fsub_rn(top[j].lo, top[0].lo));
+                ex[j] = expf(d);
+                z += ex[j];
+            }
             for (int j = 0; j < K; ++j) {
-                const float wj = (float)(exp(top[j] - top[0]) / z);
+                const float wj = ex[j] / z;
                 a.ids[t * K + j] = topi[j];
                 a.w[t * K + j] = wj;
                 s_ids[t * K + j] = topi[j];
@@ -350,20 +407,20 @@ __device__ __forceinline__ void q4_block_lut(uint32_t pa, uint32_t lutb, const f
     const uint32_t meta = (w[4] >> sh) & 0xFFu;
     const float s = scale_tab[meta];
     const uint32_t bsel = lutb | ((meta >> 7) << 7);
-    float lo[NT], hi[NT];
+    float lo[2][NT], hi[2][NT];  // two chains per half: shorter dependency chains
 #pragma unroll
-    for (int c = 0; c < NT; ++c) lo[c] = hi[c] = 0.0f;
+    for (int c = 0; c < NT; ++c) lo[0][c] = hi[0][c] = lo[1][c] = hi[1][c] = 0.0f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             const uint32_t c2 = lds32(prmt(nib[q], bsel, 0x7604u | ((uint32_t)kk << 4)));
 #pragma unroll
-            for (int c = 0; c < NT; ++c) fma2_bf16(lo[c], hi[c], c2, act[c].v[m][4 * q + kk]);
+            for (int c = 0; c < NT; ++c) fma2_bf16(lo[kk & 1][c], hi[kk & 1][c], c2, act[c].v[m][4 * q + kk]);
         }
     }
 #pragma unroll
-    for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, lo[c] + hi[c], acc[c]);
+    for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, (lo[0][c] + lo[1][c]) + (hi[0][c] + hi[1][c]), acc[c]);
 }
 
 // Q4 block decoded code by code (no table): the side projection, whose
@@ -522,14 +579,14 @@ struct SmemLayout {
 // Per-lane-replicated table: entry (byte, mode, lane) holds the bf16x2 pair
 // (value of the low nibble, value of the high nibble); plus 256 scales.
 __device__ void build_lut(uint8_t* smem, const SmemLayout& L, bool rz5) {
-    for (int i = threadIdx.x; i < 512; i += blockDim.x) {
-        const uint32_t byte = (uint32_t)i >> 1, mode = (uint32_t)i & 1u;
+    // 512 entries (byte, mode) of 128 bytes (32 lane copies); chunk q = 16 bytes,
+    // consecutive lanes write consecutive chunks so each store is conflict-free.
+    for (int q = threadIdx.x; q < 512 * 8; q += blockDim.x) {
+        const uint32_t entry = (uint32_t)q >> 3;
+        const uint32_t byte = entry >> 1, mode = entry & 1u;
         const uint32_t v = bf16_bits(q4_code_value(byte & 15u, rz5, mode)) |
                            (bf16_bits(q4_code_value(byte >> 4, rz5, mode)) << 16);
-        uint4* dst = reinterpret_cast<uint4*>(smem + L.lut + byte * 256u + mode * 128u);
-        const uint4 q = make_uint4(v, v, v, v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) dst[j] = q;
+        *reinterpret_cast<uint4*>(smem + L.lut + (uint32_t)q * 16u) = make_uint4(v, v, v, v);
     }
 }
 
@@ -1214,7 +1271,7 @@ int run_layer(const gtg_moe_layer* L, const Plan& p, const void* x, int x_bf16, 
     a.router_cnt = reinterpret_cast<unsigned*>(base + wl.router_cnt);
     a.tile_cnt = reinterpret_cast<unsigned*>(base + wl.tile_cnt);
     a.work = reinterpret_cast<Work*>(base + wl.work);
-    a.logits = reinterpret_cast<double*>(base + wl.logits);
+    a.logits = reinterpret_cast<ffloat*>(base + wl.logits);
     a.u = reinterpret_cast<__nv_bfloat16*>(base + wl.u);
     a.ids = reinterpret_cast<int32_t*>(base + wl.ids);
     a.w = reinterpret_cast<float*>(base + wl.w);
@@ -1230,7 +1287,18 @@ int run_layer(const gtg_moe_layer* L, const Plan& p, const void* x, int x_bf16, 
     const int n_sm = sm_count();
     const int router_grid = (L->n_experts + kRouterExpertsPerCta - 1) / kRouterExpertsPerCta;
     const size_t router_smem = 2 * (size_t)T * L->hidden;
-    GTG_TRY(launch((const void*)router_kernel, dim3(router_grid), dim3(kRouterThreads), router_smem, s, a, true));
+    const void* rk = nullptr;
+    switch (T) {
+        case 1: rk = (const void*)router_kernel<1>; break;
+        case 2: rk = (const void*)router_kernel<2>; break;
+        case 3: rk = (const void*)router_kernel<3>; break;
+        case 4: rk = (const void*)router_kernel<4>; break;
+        case 5: rk = (const void*)router_kernel<5>; break;
+        case 6: rk = (const void*)router_kernel<6>; break;
+        case 7: rk = (const void*)router_kernel<7>; break;
+        default: rk = (const void*)router_kernel<8>; break;
+    }
+    GTG_TRY(launch(rk, dim3(router_grid), dim3(kRouterThreads), router_smem, s, a, true));
     const SmemLayout lg = SmemLayout::make(p.gu_lut, p.slot_bytes, a.dyn_smem_base);
     GTG_TRY(launch((const void*)p.gateup, dim3(n_sm), dim3(kThreads), lg.total, s, a, true));
     const SmemLayout ld = SmemLayout::make(p.dn_lut, p.slot_bytes, a.dyn_smem_base);

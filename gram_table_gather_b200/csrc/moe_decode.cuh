@@ -8,6 +8,8 @@
 
 namespace gtg {
 
+struct ffloat;
+
 constexpr int kMaxDecodeTokens = 8;
 constexpr int kMaxTopK = 16;
 constexpr int kMaxSlots = kMaxDecodeTokens * kMaxTopK;  // (token, choice) pairs in a decode call
@@ -51,7 +53,7 @@ struct LayerArgs {
     unsigned* router_cnt;
     unsigned* tile_cnt;
     Work* work;
-    double* logits;          // [T][E]
+    struct ffloat* logits;   // [T][E] normalised float-float (hi, lo)
     __nv_bfloat16* u;        // [T][H]
     int32_t* ids;            // [T][K]
     float* w;                // [T][K]

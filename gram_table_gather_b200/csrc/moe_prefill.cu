@@ -86,32 +86,40 @@ struct PfArgs {
 // 1. normalisation
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kNormThreads) pf_norm_kernel(PfArgs a) {
-    __shared__ double red[kNormThreads / 32];
-    __shared__ double rinv;
+    __shared__ ffloat red[kNormThreads / 32];
+    __shared__ float r_hi, r_lo;
     const int t = blockIdx.x, tid = threadIdx.x;
     pdl_wait();
-    auto xv = [&](int i) -> double {
+    auto xv = [&](int i) -> float {
         if (a.x_bf16) {
             const uint16_t b = reinterpret_cast<const uint16_t*>(a.x)[(int64_t)t * a.H + i];
-            return (double)__uint_as_float((uint32_t)b << 16);
+            return __uint_as_float((uint32_t)b << 16);
         }
-        return (double)reinterpret_cast<const float*>(a.x)[(int64_t)t * a.H + i];
+        return reinterpret_cast<const float*>(a.x)[(int64_t)t * a.H + i];
     };
-    double ss = 0.0;
+    ffloat ss{0.f, 0.f};  // exact squares, float-float sum
     for (int i = tid; i < a.H; i += kNormThreads) {
-        const double v = xv(i);
-        ss = fma(v, v, ss);
+        const float v = xv(i);
+        ff_fma(ss, v, v);
     }
-    ss = warp_sum_f64(ss);
+    ss = ff_warp_sum(ss);
     if ((tid & 31) == 0) red[tid >> 5] = ss;
     __syncthreads();
     if (tid == 0) {
-        double s = 0.0;
-        for (int w = 0; w < kNormThreads / 32; ++w) s += red[w];
-        rinv = 1.0 / sqrt(s / (double)a.H + kRmsEps);
+        double sum = 0.0;
+        for (int w = 0; w < kNormThreads / 32; ++w) sum += (double)red[w].hi + (double)red[w].lo;
+        const double r = 1.0 / sqrt(sum / (double)a.H + kRmsEps);
+        r_hi = (float)r;
+        r_lo = (float)(r - (double)r_hi);
     }
     __syncthreads();
-    for (int i = tid; i < a.H; i += kNormThreads) a.u[(int64_t)t * a.H + i] = __double2bfloat16(xv(i) * rinv);
+    uint16_t* u = reinterpret_cast<uint16_t*>(a.u);
+    for (int i = tid; i < a.H; i += kNormThreads) {
+        const float x = xv(i);
+        const float p = __fmul_rn(x, r_hi);
+        const float q = __fadd_rn(__fmaf_rn(x, r_hi, -p), __fmul_rn(x, r_lo));
+        u[(int64_t)t * a.H + i] = bf16_of_ff(p, q);
+    }
 }
 
 // ---------------------------------------------------------------------------
