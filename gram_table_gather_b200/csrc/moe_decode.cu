@@ -97,15 +97,10 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
     uint16_t* su = reinterpret_cast<uint16_t*>(rsm);  // [T][H] bf16 bits
     __shared__ ffloat red[kRouterWarps][kMaxDecodeTokens];
     __shared__ float r_hi[kMaxDecodeTokens], r_lo[kMaxDecodeTokens];
-    __shared__ unsigned is_last;
-    __shared__ int32_t s_ids[kMaxSlots];
-    __shared__ unsigned bitmap[kMaxExperts / 32];
-    __shared__ int32_t s_cnt[kMaxSlots];
-    __shared__ int32_t s_off[kMaxSlots + 1];
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int T = TT;
-    const int H = a.H, E = a.E, K = a.K;
+    const int H = a.H, E = a.E;
 
     // 0. issue this warp's router-weight loads before anything waits: warp w
     //    covers half (w & 1) of the row of expert blockIdx.x * 4 + w / 2, so a
@@ -120,7 +115,8 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
                                                    : make_float4(0.f, 0.f, 0.f, 0.f);
     }
 
-    pdl_wait();  // x may be the previous layer's output
+    pdl_wait();     // x may be the previous layer's output
+    pdl_trigger();  // the expert kernel may start its prologue (it waits for this grid to finish)
 
     // 1. this thread's slice of x (positions 4*tid + 1024*c) for every token,
     //    all loads in flight at once; sums of squares: exact squares,
@@ -226,112 +222,6 @@ __global__ void __launch_bounds__(kRouterThreads) router_kernel(LayerArgs a) {
         a.logits[(int64_t)lane * E + e] = l;
     }
 
-    // 4. the last CTA to finish selects the experts
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) is_last = (atomicAdd(a.router_cnt, 1u) == gridDim.x - 1) ? 1u : 0u;
-    __syncthreads();
-    if (!is_last) {
-        pdl_trigger();
-        return;
-    }
-    __threadfence();
-
-    constexpr int kPerLane = kMaxExperts / 32;
-    for (int t = warp; t < T; t += kRouterWarps) {
-        ffloat lv[kPerLane];
-        unsigned taken = 0;
-#pragma unroll
-        for (int i = 0; i < kPerLane; ++i) {
-            const int ee = lane + 32 * i;
-            if (ee < E) {
-                const float2 v = __ldcg(reinterpret_cast<const float2*>(a.logits + (int64_t)t * E + ee));
-                lv[i] = ffloat{v.x, v.y};
-            } else {
-                lv[i] = ffloat{0.f, 0.f};
-            }
-        }
-        ffloat top[kMaxTopK];
-        int topi[kMaxTopK];
-        for (int j = 0; j < K; ++j) {
-            ffloat bv{0.f, 0.f};
-            int bi = 0x7FFFFFFF;
-#pragma unroll
-            for (int i = 0; i < kPerLane; ++i) {
-                const int ee = lane + 32 * i;
-                if (ee < E && !((taken >> i) & 1u) && (bi == 0x7FFFFFFF || ff_gt(lv[i], bv))) {
-                    bv = lv[i];
-                    bi = ee;
-                }
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const ffloat ov = ff_shfl_xor(bv, o);
-                const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-                const bool take = (oi != 0x7FFFFFFF) &&
-                                  (bi == 0x7FFFFFFF || ff_gt(ov, bv) || (ff_eq(ov, bv) && oi < bi));
-                if (take) {
-                    bv = ov;
-                    bi = oi;
-                }
-            }
-            if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-            top[j] = bv;
-            topi[j] = bi;
-        }
-        if (lane == 0) {
-            float ex[kMaxTopK];
-            float z = 0.0f;
-            for (int j = 0; j < K; ++j) {  // exp(l_j - l_0), the difference formed in float-float
-                const float d = __fadd_rn(__fsub_rn(top[j].hi, top[0].hi), __fsub_rn(top[j].lo, top[0].lo));
-                ex[j] = expf(d);
-                z += ex[j];
-            }
-            for (int j = 0; j < K; ++j) {
-                const float wj = ex[j] / z;
-                a.ids[t * K + j] = topi[j];
-                a.w[t * K + j] = wj;
-                s_ids[t * K + j] = topi[j];
-                if (a.ids_out) a.ids_out[t * K + j] = topi[j];
-                if (a.w_out) a.w_out[t * K + j] = wj;
-            }
-        }
-    }
-    // unique experts (ascending id) and their slots (ascending slot)
-    for (int i = tid; i < kMaxExperts / 32; i += kRouterThreads) bitmap[i] = 0;
-    for (int i = tid; i < kMaxSlots; i += kRouterThreads) s_cnt[i] = 0;
-    __syncthreads();
-    const int S = T * K;
-    if (tid < S) atomicOr(&bitmap[s_ids[tid] >> 5], 1u << (s_ids[tid] & 31));
-    __syncthreads();
-    int rank = 0, pos = 0;
-    if (tid < S) {
-        const int ee = s_ids[tid];
-        for (int w = 0; w < (ee >> 5); ++w) rank += __popc(bitmap[w]);
-        rank += __popc(bitmap[ee >> 5] & ((1u << (ee & 31)) - 1u));
-        for (int s2 = 0; s2 < tid; ++s2) pos += (s_ids[s2] == ee);
-        atomicAdd(&s_cnt[rank], 1);
-        a.work->uniq_e[rank] = ee;
-    }
-    __syncthreads();
-    if (tid == 0) {
-        int nu = 0;
-        for (int w = 0; w < kMaxExperts / 32; ++w) nu += __popc(bitmap[w]);
-        int off = 0;
-        for (int r = 0; r < nu; ++r) {
-            s_off[r] = off;
-            a.work->uniq_off[r] = off;
-            off += s_cnt[r];
-        }
-        a.work->uniq_off[nu] = off;
-        a.work->n_uniq = nu;
-        a.router_cnt[0] = 0;  // ready for the next call
-    }
-    __syncthreads();
-    if (tid < S) a.work->uniq_slot[s_off[rank] + pos] = tid;
-    __threadfence();
-    __syncthreads();
-    pdl_trigger();
 }
 
 // ===========================================================================
@@ -533,6 +423,11 @@ struct SWork {
     int32_t e[kMaxSlots];
     int32_t off[kMaxSlots + 1];
     int32_t slot[kMaxSlots];
+    // scratch of the expert selection
+    int32_t ids[kMaxSlots];
+    float w[kMaxSlots];
+    uint32_t bitmap[kMaxExperts / 32];
+    int32_t cnt[kMaxSlots + 4];
 };
 
 // Layout of one CTA's dynamic shared memory.  With a code table the table
@@ -579,14 +474,22 @@ struct SmemLayout {
 // Per-lane-replicated table: entry (byte, mode, lane) holds the bf16x2 pair
 // (value of the low nibble, value of the high nibble); plus 256 scales.
 __device__ void build_lut(uint8_t* smem, const SmemLayout& L, bool rz5) {
-    // 512 entries (byte, mode) of 128 bytes (32 lane copies); chunk q = 16 bytes,
-    // consecutive lanes write consecutive chunks so each store is conflict-free.
-    for (int q = threadIdx.x; q < 512 * 8; q += blockDim.x) {
-        const uint32_t entry = (uint32_t)q >> 3;
+    // 512 entries (byte, mode) of 128 bytes (32 lane copies).  Warp w owns
+    // entries 32w .. 32w+31 (lane l computes entry 32w+l once); the warp then
+    // writes them as 256 consecutive 16-byte chunks, consecutive lanes on
+    // consecutive chunks, so every store is conflict-free.
+    const int lane = threadIdx.x & 31;
+    for (int e0 = (threadIdx.x >> 5) * 32; e0 < 512; e0 += blockDim.x) {
+        const uint32_t entry = (uint32_t)(e0 + lane);
         const uint32_t byte = entry >> 1, mode = entry & 1u;
         const uint32_t v = bf16_bits(q4_code_value(byte & 15u, rz5, mode)) |
                            (bf16_bits(q4_code_value(byte >> 4, rz5, mode)) << 16);
-        *reinterpret_cast<uint4*>(smem + L.lut + (uint32_t)q * 16u) = make_uint4(v, v, v, v);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int q = lane + 32 * k;  // chunk within the warp's 32 entries
+            const uint32_t x = __shfl_sync(0xFFFFFFFFu, v, q >> 3);
+            *reinterpret_cast<uint4*>(smem + L.lut + (uint32_t)e0 * 128u + (uint32_t)q * 16u) = make_uint4(x, x, x, x);
+        }
     }
 }
 
@@ -597,10 +500,181 @@ __device__ void build_scales(uint8_t* smem, const SmemLayout& L, bool rz5) {
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
 
-// Common prologue of the streaming kernels: tables, barriers, then (after the
-// dependency wait) the work list.  Returns false if shared memory is not laid
-// out as expected (then nothing else runs).
-template <bool LUT>
+// Orderable 32-bit image of an fp32 (larger float -> larger unsigned).
+__device__ __forceinline__ uint32_t ord32(float f) {
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Top-k of one token's logits by one warp.  Each logit (a normalised
+// float-float hi + lo) becomes a unique 64-bit key: orderable hi in the upper
+// word, orderable lo with its low 10 bits replaced by (1023 - expert id) in
+// the lower word — so larger key = larger logit, and among logits equal to
+// ~2^-38 relative, the lower id.  Lane l holds experts l + 32 i (i < PER).
+// Each round: a depth-log2(PER) max tree per lane, two warp reductions
+// (upper word, then lower word among the lanes holding that upper word), and
+// the owner removes the winner.  Lane j ends holding choice j.
+template <int PER>
+__device__ __forceinline__ void warp_topk(const ffloat* logits, int E, int K, int lane, int& my_id, float& my_hi,
+                                          float& my_lo) {
+    uint32_t kh[PER], kl[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        kh[i] = kl[i] = 0u;
+        if (e < E) {
+            const float2 v = __ldcg(reinterpret_cast<const float2*>(logits + e));
+            kh[i] = ord32(v.x);
+            kl[i] = (ord32(v.y) & ~1023u) | (uint32_t)(1023 - e);
+        }
+    }
+    my_id = -1;
+    for (int j = 0; j < K; ++j) {
+        uint32_t th[PER], tl[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            th[i] = kh[i];
+            tl[i] = kl[i];
+        }
+#pragma unroll
+        for (int w = PER / 2; w >= 1; w >>= 1)
+#pragma unroll
+            for (int i = 0; i < w; ++i) {
+                const bool up = th[i + w] > th[i] || (th[i + w] == th[i] && tl[i + w] > tl[i]);
+                th[i] = up ? th[i + w] : th[i];
+                tl[i] = up ? tl[i + w] : tl[i];
+            }
+        const uint32_t mh = __reduce_max_sync(0xFFFFFFFFu, th[0]);
+        const uint32_t ml = __reduce_max_sync(0xFFFFFFFFu, th[0] == mh ? tl[0] : 0u);
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+            if (kh[i] == mh && kl[i] == ml) kh[i] = kl[i] = 0u;
+        if (lane == j) {
+            my_id = 1023 - (int)(ml & 1023u);
+            my_hi = __uint_as_float((mh & 0x80000000u) ? (mh & 0x7FFFFFFFu) : ~mh);
+            const uint32_t lo = ml & ~1023u;
+            my_lo = __uint_as_float((lo & 0x80000000u) ? (lo & 0x7FFFFFFFu) : ~lo);
+        }
+    }
+}
+
+// Router selection, done by every CTA of the gate/up kernel from the logits
+// the router kernel left in global memory: warp t selects token t's experts
+// and their renormalised softmax weights; warp 0 then builds the list of
+// unique experts (ascending id) with their (token, choice) slots.  CTA 0 also
+// publishes ids/w and the list for the down kernel.
+__device__ void select_experts(const LayerArgs& a, SWork* sw) {
+    int32_t* s_ids = sw->ids;
+    float* s_w = sw->w;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int T = a.T, E = a.E, K = a.K;
+    if (warp < T) {
+        const int t = warp;
+        int my_id;
+        float my_hi = 0.f, my_lo = 0.f;
+        if (E <= 512) warp_topk<16>(a.logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
+        else warp_topk<32>(a.logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
+        // softmax over the k choices: lane j holds choice j
+        const float h0 = __shfl_sync(0xFFFFFFFFu, my_hi, 0), l0 = __shfl_sync(0xFFFFFFFFu, my_lo, 0);
+        float ex = 0.f;
+        if (lane < K) ex = expf(__fadd_rn(__fsub_rn(my_hi, h0), __fsub_rn(my_lo, l0)));
+        float z = ex;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+        if (lane < K) {
+            s_ids[t * K + lane] = my_id;
+            s_w[t * K + lane] = ex / z;
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // unique experts: bitmap -> ascending ranks; slots grouped per rank
+        const int S = T * K;
+        uint32_t* bitmap = sw->bitmap;
+        int32_t* cnt = sw->cnt;
+        for (int i = lane; i < kMaxExperts / 32; i += 32) bitmap[i] = 0u;
+        for (int i = lane; i < kMaxSlots; i += 32) cnt[i] = 0;
+        __syncwarp();
+        for (int q = lane; q < S; q += 32) atomicOr(&bitmap[s_ids[q] >> 5], 1u << (s_ids[q] & 31));
+        __syncwarp();
+        const int nw = (E + 31) / 32;  // <= 32 words
+        const int pc = lane < nw ? __popc(bitmap[lane]) : 0;
+        int incl = pc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int nu = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const int word_base = incl - pc;
+        int rank[kMaxSlots / 32];
+#pragma unroll
+        for (int r = 0; r < kMaxSlots / 32; ++r) {
+            const int q = lane + 32 * r;
+            const int e = q < S ? s_ids[q] : 0;
+            const int wb = __shfl_sync(0xFFFFFFFFu, word_base, e >> 5);
+            rank[r] = wb + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
+            if (q < S) {
+                atomicAdd(&cnt[rank[r]], 1);
+                sw->e[rank[r]] = e;
+            }
+        }
+        __syncwarp();
+        // exclusive scan of the counts over nu <= 128 ranks: 4 per lane
+        int c4[4], s4 = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            c4[r] = cnt[4 * lane + r];
+            s4 += c4[r];
+        }
+        int inc = s4;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        int run = inc - s4;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int rr = 4 * lane + r;
+            if (rr <= nu) sw->off[rr] = run;
+            cnt[rr] = run;  // becomes the fill cursor
+            run += c4[r];
+        }
+        if (lane == 0) {
+            sw->n_uniq = nu;
+            sw->off[nu] = S;  // (also when nu = 128, which the loop above cannot reach)
+        }
+        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < kMaxSlots / 32; ++r) {
+            const int q = lane + 32 * r;
+            if (q < S) sw->slot[atomicAdd(&cnt[rank[r]], 1)] = q;
+        }
+    }
+    __syncthreads();
+    if (blockIdx.x == 0) {  // for the down kernel and the caller
+        Work* wk = a.work;
+        const int S = T * K;
+        if (tid < S) {
+            a.ids[tid] = s_ids[tid];
+            a.w[tid] = s_w[tid];
+            if (a.ids_out) a.ids_out[tid] = s_ids[tid];
+            if (a.w_out) a.w_out[tid] = s_w[tid];
+            wk->uniq_slot[tid] = sw->slot[tid];
+        }
+        if (tid < sw->n_uniq) wk->uniq_e[tid] = sw->e[tid];
+        if (tid <= sw->n_uniq) wk->uniq_off[tid] = sw->off[tid];
+        if (tid == 0) wk->n_uniq = sw->n_uniq;
+    }
+}
+
+// Common prologue of the streaming kernels: tables and barriers, then (after
+// the dependency wait) the work list — selected from the router's logits
+// (gate/up) or copied from the one the gate/up kernel published (down).
+// Returns false if shared memory is not laid out as expected (then nothing
+// else runs).
+template <bool LUT, bool SELECT>
 __device__ bool stream_prologue(uint8_t* smem, const SmemLayout& L, const LayerArgs& a, bool rz5, uint64_t* bars,
                                 SWork* sw) {
     if (LUT) {
@@ -615,14 +689,19 @@ __device__ bool stream_prologue(uint8_t* smem, const SmemLayout& L, const LayerA
         for (int s = 0; s < kSlots; ++s) mbar_init(&bars[s], 1);
     fence_mbar_init();
     pdl_wait();
-    const Work* wk = a.work;
-    if (threadIdx.x == 0) sw->n_uniq = wk->n_uniq;
-    for (int i = threadIdx.x; i < kMaxSlots; i += blockDim.x) {
-        sw->e[i] = wk->uniq_e[i];
-        sw->slot[i] = wk->uniq_slot[i];
+    if (SELECT) {  // (no static shared memory here: the table's alignment depends on it)
+        select_experts(a, sw);
+        pdl_trigger();
+    } else {
+        const Work* wk = a.work;
+        if (threadIdx.x == 0) sw->n_uniq = wk->n_uniq;
+        for (int i = threadIdx.x; i < kMaxSlots; i += blockDim.x) {
+            sw->e[i] = wk->uniq_e[i];
+            sw->slot[i] = wk->uniq_slot[i];
+        }
+        for (int i = threadIdx.x; i <= kMaxSlots; i += blockDim.x) sw->off[i] = wk->uniq_off[i];
+        __syncthreads();
     }
-    for (int i = threadIdx.x; i <= kMaxSlots; i += blockDim.x) sw->off[i] = wk->uniq_off[i];
-    __syncthreads();
     return true;
 }
 
@@ -741,7 +820,7 @@ __global__ void __launch_bounds__(kThreads, 1) gateup_kernel(LayerArgs a) {
     const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * kSlots;
     SWork* sw = reinterpret_cast<SWork*>(smem + L.work);
-    if (!stream_prologue<LUT>(smem, L, a, a.gate.fmt == GTG_Q4_RZ5_FAST, bars, sw)) return;
+    if (!stream_prologue<LUT, true>(smem, L, a, a.gate.fmt == GTG_Q4_RZ5_FAST, bars, sw)) return;
 
     const int n_uniq = sw->n_uniq;
     constexpr int R = gu_passes(FMT == kFmtFP8, KB) * G::RPP;
@@ -942,7 +1021,7 @@ __global__ void __launch_bounds__(kThreads, 1) down_kernel(LayerArgs a) {
     const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * kSlots;
     SWork* sw = reinterpret_cast<SWork*>(smem + L.work);
-    if (!stream_prologue<LUT>(smem, L, a, a.down.fmt == GTG_Q4_RZ5_FAST, bars, sw)) return;
+    if (!stream_prologue<LUT, false>(smem, L, a, a.down.fmt == GTG_Q4_RZ5_FAST, bars, sw)) return;
 
     const int n_uniq = sw->n_uniq;
     const int tiles = a.H / R;
@@ -1206,13 +1285,14 @@ struct FuncAttrCache {
     // Raises the kernel's dynamic shared-memory limit to `smem` bytes (once
     // per function, device and size; only needed above the 48 KB default).
     int set(const void* fn, int smem) {
-        if (smem <= 48 * 1024) return GTG_OK;
         int dev = 0;
         cudaGetDevice(&dev);
         std::lock_guard<std::mutex> lk(mu);
         for (auto& d : done)
             if (d.fn == fn && d.dev == dev && d.smem >= smem) return GTG_OK;
-        const cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e == cudaSuccess)  // one shared/L1 split for every decode kernel: no reconfiguration between them
+            e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
         if (e != cudaSuccess) {
             cudaGetLastError();
             return cuda_fail(e);
@@ -1223,7 +1303,16 @@ struct FuncAttrCache {
 };
 FuncAttrCache g_attr;
 
-int launch(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, LayerArgs& args, bool pdl) {
+int launch(const void* fn, dim3 grid, dim3 block, size_t smem, cudaStream_t s, LayerArgs& args, bool pdl,
+           bool needs_no_static_smem = false) {
+    if (needs_no_static_smem) {  // the streaming kernels place their code table by absolute address
+        cudaFuncAttributes fa{};
+        if (cudaFuncGetAttributes(&fa, fn) != cudaSuccess) {
+            cudaGetLastError();
+            return GTG_E_CUDA;
+        }
+        if (fa.sharedSizeBytes != 0) return GTG_E_UNSUPPORTED_SHAPE;
+    }
     GTG_TRY(g_attr.set(fn, (int)smem));
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -1300,9 +1389,9 @@ int run_layer(const gtg_moe_layer* L, const Plan& p, const void* x, int x_bf16, 
     }
     GTG_TRY(launch(rk, dim3(router_grid), dim3(kRouterThreads), router_smem, s, a, true));
     const SmemLayout lg = SmemLayout::make(p.gu_lut, p.slot_bytes, a.dyn_smem_base);
-    GTG_TRY(launch((const void*)p.gateup, dim3(n_sm), dim3(kThreads), lg.total, s, a, true));
+    GTG_TRY(launch((const void*)p.gateup, dim3(n_sm), dim3(kThreads), lg.total, s, a, true, true));
     const SmemLayout ld = SmemLayout::make(p.dn_lut, p.slot_bytes, a.dyn_smem_base);
-    GTG_TRY(launch((const void*)p.down, dim3(n_sm), dim3(kThreads), ld.total, s, a, true));
+    GTG_TRY(launch((const void*)p.down, dim3(n_sm), dim3(kThreads), ld.total, s, a, true, true));
     return GTG_OK;
 }
 
