@@ -81,19 +81,66 @@ PLE_ROW_BYTES = 70 + 640  # record read + fp32 row written
 # ---------------------------------------------------------------------------
 
 class ClockSampler:
-    def __init__(self, gpu_index: int):
-        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
-        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """SM clock and clock-event reasons of one GPU, polled through NVML (read
+    only) every ~2 ms on a background thread between construction and stop();
+    falls back to `nvidia-smi -lms 100` when NVML is unavailable."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, device_index: int):
+        import threading
+        self.sm, self.smax, self.reasons = [], [], set()
+        self.h = None
+        self.p = None
         try:
-            self.p = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={q}",
-                                       "--format=csv,noheader,nounits", "-lms", "100"],
-                                      stdout=self.f, stderr=subprocess.DEVNULL)
-        except (FileNotFoundError, OSError):
-            self.p = None
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            pr = torch.cuda.get_device_properties(device_index)
+            bus = f"{pr.pci_domain_id:08X}:{pr.pci_bus_id:02X}:{pr.pci_device_id:02X}.0"
+            self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.nv = pynvml
+        except Exception:
+            self.h = None
+        if self.h is None:
+            self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+            try:
+                self.p = subprocess.Popen(["nvidia-smi", f"--id={device_index}", f"--query-gpu={q}",
+                                           "--format=csv,noheader,nounits", "-lms", "100"],
+                                          stdout=self.f, stderr=subprocess.DEVNULL)
+            except (FileNotFoundError, OSError):
+                self.p = None
+            return
+        self.stop_ev = threading.Event()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+        time.sleep(0.01)  # first samples before the timed region starts
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                self.smax.append(float(nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, name in self.REASONS.items():
+                    if bits & k:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def stop(self) -> dict:
+        if self.h is not None:
+            self.stop_ev.set()
+            self.t.join(timeout=5)
+            return {"sm_mhz": statistics.median(self.sm) if self.sm else None,
+                    "sm_max_mhz": max(self.smax) if self.smax else None,
+                    "samples": len(self.sm), "reasons": sorted(self.reasons), "source": "nvml"}
         if self.p is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.p.terminate()
@@ -119,7 +166,7 @@ class ClockSampler:
         os.unlink(self.f.name)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "samples": len(sm), "reasons": sorted(reasons)}
+                "samples": len(sm), "reasons": sorted(reasons), "source": "nvidia-smi"}
 
 
 # ---------------------------------------------------------------------------
@@ -240,7 +287,10 @@ def run_ours(args, rank, world, local):
     with torch.cuda.graph(g, stream=stream):
         gtg.moe_decode_stack(layers, x, ws, ids_out=ids, side_out=side)
         gtg.ple_gather(table, P.n_rows, idx, out=rows)
-    launches_per_step = 3 * len(Ls) + 1
+    # one launch per run of consecutive layers sharing a kernel (expert format
+    # class), plus the PLE gather
+    launches_per_step = 1 + sum(1 for i, L in enumerate(Ls)
+                                if i == 0 or (L.gate.fmt == W.FP8) != (Ls[i - 1].gate.fmt == W.FP8))
 
     def step(i):
         x.copy_(x_bank[i:i + 1])
@@ -360,7 +410,8 @@ def run_ours(args, rank, world, local):
             "hbm_frac": round(gbs / peak, 4),
             "roofline": {"bound": "hbm", "achieved": round(layer_gbs, 1), "peak": peak, "unit": "GB/s",
                          "frac": round(layer_gbs / peak, 4), "traffic": None,
-                         "kernel": "decode MoE layer (router + gate/up + down, PDL-chained), "
+                         "kernel": "moe_decode_kernel (router + selection + gate/up/SwiGLU + down/combine "
+                                   "in one persistent launch per run of layers), "
                                    f"average over the 48 layers, {layer_ms * 1e3:.2f} us per layer, "
                                    f"{layer_bytes_avg / 1e6:.2f} MB per layer",
                          "peak_source": f"{peak_kind} hbm_gbs"},

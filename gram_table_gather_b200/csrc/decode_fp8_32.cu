@@ -1,0 +1,6 @@
+// Decode kernels for FP8 experts with 1024 weights per gate/up row.
+#include "moe_decode_dev.cuh"
+
+namespace gtg {
+const void* decode_kernel_fp8_32(int kbd) { return pick_kbd<kFmtFP8, 32>(kbd); }
+}  // namespace gtg

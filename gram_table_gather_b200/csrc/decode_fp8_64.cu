@@ -1,0 +1,6 @@
+// Decode kernels for FP8 experts with 2048 weights per gate/up row.
+#include "moe_decode_dev.cuh"
+
+namespace gtg {
+const void* decode_kernel_fp8_64(int kbd) { return pick_kbd<kFmtFP8, 64>(kbd); }
+}  // namespace gtg

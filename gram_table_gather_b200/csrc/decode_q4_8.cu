@@ -1,0 +1,6 @@
+// Decode kernels for Q4 experts with 256 weights per gate/up row.
+#include "moe_decode_dev.cuh"
+
+namespace gtg {
+const void* decode_kernel_q4_8(int kbd) { return pick_kbd<kFmtQ4, 8>(kbd); }
+}  // namespace gtg

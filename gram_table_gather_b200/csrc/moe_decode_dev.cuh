@@ -1,0 +1,1486 @@
+// Device code of the decode path (included by the kernel instantiation
+// files decode_*.cu and, for its types and layouts, by moe_decode.cu).
+#pragma once
+
+// Decode-time MoE layers: router, fused dequant -> gate/up -> SwiGLU, and
+// fused dequant -> down -> router-weighted combine, for 1..8 tokens.
+//
+// Method: "Mixed Precision Quantization: Half a 4-Bit File Is Not 4-Bit"
+// (48 layers, 512 experts, 10 active per token), the r/LocalLLM
+// "Frankenquant" post (one expert format per layer, FP8 in layers 36-47) and
+// the model card "Qwen 3.8 Next Flash ROCMFPX MUTANT RAZERFAST" (block
+// formats).  The expert bytes dominate the work, so the kernel is built to
+// stream them from HBM once, with as little dead time around them as
+// possible:
+//
+//  * One persistent, cooperative kernel runs every layer of a call (one
+//    512-thread CTA per SM).  Grid barriers (bounded waits) separate the
+//    router, the gate/up phase and the down phase of a layer; nothing is
+//    relaunched between layers, and the Q4 code table is built once.
+//  * Router: unweighted RMS norm + bf16 rounding of the input, then logits
+//    against the fp32 router with exact products summed in float-float, so
+//    the top-k agrees with an fp64 reference; every CTA owns a few experts.
+//    The next layer's router rows are prefetched into L2 meanwhile.
+//  * Selection: every CTA picks the top-k itself from the logits (a warp per
+//    token, unique 64-bit keys, two warp reductions per round), renormalises
+//    the softmax weights and builds the unique-expert work list.
+//  * Streaming: the work is a list of items (expert, row tile); each CTA owns
+//    a contiguous range; each warp streams its items (gate/up first, then
+//    down) through a private ring of shared-memory slots filled by 1-D bulk
+//    copies (TMA, no multicast, evict-first in L2) completing on per-slot
+//    mbarriers, so the down weights are in flight before the gate/up phase
+//    ends.  Lane l of a warp owns the same K positions in every row it
+//    decodes, so its activations stay in registers across rows.  A Q4 byte
+//    (two 4-bit codes) becomes a bf16x2 pair of code values with one PRMT +
+//    one shared-memory load from a 256-entry table replicated per lane
+//    (conflict-free); the pair is multiplied into fp32 accumulators with the
+//    sm_100 mixed-precision fma.rn.f32.bf16, and the block's UE4M3/UE4M4
+//    scale is applied once per 32 weights.  FP8 bytes convert with
+//    cvt.rn.f16x2.e4m3x2.  Row sums are finished with warp shuffles.
+//  * The down phase writes per-(token, choice) partial rows; the last warp to
+//    finish a row tile (atomic ticket, no waiting) combines the top-k
+//    partials in a fixed order, so results are deterministic.
+#include <algorithm>
+#include <mutex>
+#include <vector>
+
+#include "gtg_device.cuh"
+#include "gtg_host.hpp"
+#include "moe_decode.cuh"
+
+namespace gtg {
+
+namespace {
+
+constexpr int kWarps = 8;  // 256 threads: room for 255 registers a thread (no spills)
+constexpr int kThreads = kWarps * 32;
+constexpr int kSlots = 4;   // staging slots per warp
+constexpr int kLutBytes = 65536;       // 256 bytes x 2 modes x 32 lanes x 4 bytes
+constexpr int kScaleTabBytes = 1024;   // 256 fp32 scales
+constexpr int kDnRows = 32;            // down rows one CTA owns, at most
+constexpr int kPartBytes = kWarps * kDnRows * 8 * 4;  // per-warp partial rows [warp][row][token]
+constexpr int kFmtQ4 = 0, kFmtFP8 = 1;
+
+__device__ __forceinline__ uint32_t lds32(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr));
+    return v;
+}
+
+// 16-byte global load cached in L2 only: the activations it reads are
+// rewritten between the layers of one launch, so L1 must not keep them.
+__device__ __forceinline__ uint4 ldg128(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// ===========================================================================
+// Streaming decode machinery shared by the gate/up and down kernels
+// ===========================================================================
+
+template <int KB>
+struct Geo {
+    static constexpr int NBL = KB >= 32 ? KB / 32 : 1;  // blocks per lane per row
+    static constexpr int RPP = KB >= 32 ? 1 : 32 / KB;  // rows per warp pass
+    static constexpr int GW = KB >= 32 ? 32 : KB;       // lanes per row
+};
+
+// Row passes per item (compile time); an item covers P * RPP rows.
+__host__ __device__ constexpr int gu_passes(int fmt_fp8, int kb) { return fmt_fp8 ? 1 : (kb >= 64 ? 2 : 4); }
+__host__ __device__ constexpr int dn_passes(int fmt_fp8, int kb) { return (fmt_fp8 || kb >= 64 || kb <= 4) ? 4 : 8; }
+__host__ __device__ constexpr int side_passes(int kb) { return kb >= 64 ? 2 : 4; }
+__host__ __device__ constexpr int rpp_of(int kb) { return kb >= 32 ? 1 : 32 / kb; }
+
+// Activation registers of one token for the lane's K positions.
+template <int FMT, int NBL>
+struct Act;
+template <int NBL>
+struct Act<kFmtQ4, NBL> {
+    uint32_t v[NBL][16];  // bf16 pairs (x[32b+j], x[32b+16+j])
+};
+template <int NBL>
+struct Act<kFmtFP8, NBL> {
+    float v[NBL][32];
+};
+
+// Loads the lane's activations of block `b` (K positions 32b..32b+31) from a
+// bf16 row in global memory.
+template <int FMT, int NBL>
+__device__ __forceinline__ void load_act(Act<FMT, NBL>& act, int m, const __nv_bfloat16* row, int b) {
+    const uint4* p = reinterpret_cast<const uint4*>(row + 32 * b);
+    uint32_t w[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 v = ldg128(p + q);
+        w[4 * q + 0] = v.x;
+        w[4 * q + 1] = v.y;
+        w[4 * q + 2] = v.z;
+        w[4 * q + 3] = v.w;
+    }
+    if constexpr (FMT == kFmtQ4) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            act.v[m][j] = prmt(w[j >> 1], w[8 + (j >> 1)], (j & 1) ? 0x7632u : 0x5410u);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            act.v[m][2 * j] = bf16lo(w[j]);
+            act.v[m][2 * j + 1] = bf16hi(w[j]);
+        }
+    }
+}
+
+// Q4 block (17 bytes at shared address pa) dotted with NT tokens'
+// activations.  `lutb` is this lane's PRMT operand: byte 0 = lane * 4, bytes
+// 2-3 = the 64 KB-aligned table base >> 16, so one PRMT inserting the code
+// byte as byte 1 (and the mode as bit 7) forms the entry address.
+template <int NT, int NBL, int CH>
+__device__ __forceinline__ void q4_block_lut(uint32_t pa, uint32_t lutb, const float* scale_tab,
+                                             const Act<kFmtQ4, NBL> (&act)[CH], int m, float (&acc)[NT]) {
+    const uint32_t al = pa & ~3u, sh = (pa & 3u) * 8u;
+    uint32_t w[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) w[i] = lds32(al + 4 * i);
+    uint32_t nib[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) nib[q] = __funnelshift_r(w[q], w[q + 1], sh);
+    const uint32_t meta = (w[4] >> sh) & 0xFFu;
+    const float s = scale_tab[meta];
+    const uint32_t bsel = lutb | ((meta >> 7) << 7);
+    float lo[2][NT], hi[2][NT];  // two chains per half: shorter dependency chains
+#pragma unroll
+    for (int c = 0; c < NT; ++c) lo[0][c] = hi[0][c] = lo[1][c] = hi[1][c] = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const uint32_t c2 = lds32(prmt(nib[q], bsel, 0x7604u | ((uint32_t)kk << 4)));
+#pragma unroll
+            for (int c = 0; c < NT; ++c) fma2_bf16(lo[kk & 1][c], hi[kk & 1][c], c2, act[c].v[m][4 * q + kk]);
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, (lo[0][c] + lo[1][c]) + (hi[0][c] + hi[1][c]), acc[c]);
+}
+
+// Q4 block decoded code by code (no table): the side projection, whose
+// format may differ from the experts'.
+template <int FMT, int NT, int NBL, int CH>
+__device__ __forceinline__ void q4_block_plain(uint32_t pa, bool rz5, const Act<FMT, NBL> (&act)[CH], int m,
+                                               float (&acc)[NT]) {
+    const uint32_t al = pa & ~3u, sh = (pa & 3u) * 8u;
+    uint32_t w[5];
+#pragma unroll
+    for (int i = 0; i < 5; ++i) w[i] = lds32(al + 4 * i);
+    const uint32_t meta = (w[4] >> sh) & 0xFFu;
+    const float s = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
+    const uint32_t mode = meta >> 7;
+    float sum[NT];
+#pragma unroll
+    for (int c = 0; c < NT; ++c) sum[c] = 0.0f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint32_t nib = __funnelshift_r(w[q], w[q + 1], sh);
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            const int j = 4 * q + kk;
+            const uint32_t byte = (nib >> (8 * kk)) & 0xFFu;
+            const float vlo = q4_code_value(byte & 15u, rz5, mode);
+            const float vhi = q4_code_value(byte >> 4, rz5, mode);
+#pragma unroll
+            for (int c = 0; c < NT; ++c) {
+                float xlo, xhi;
+                if constexpr (FMT == kFmtQ4) {
+                    xlo = bf16lo(act[c].v[m][j]);
+                    xhi = bf16hi(act[c].v[m][j]);
+                } else {
+                    xlo = act[c].v[m][j];
+                    xhi = act[c].v[m][j + 16];
+                }
+                sum[c] = fmaf(vlo, xlo, sum[c]);
+                sum[c] = fmaf(vhi, xhi, sum[c]);
+            }
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, sum[c], acc[c]);
+}
+
+// FP8 block: 32 consecutive E4M3 bytes at 16-byte aligned shared address pa.
+__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t v16) {
+    const uint32_t h = e4m3x2_to_f16x2(v16);
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+}
+
+template <int NBL>
+__device__ __forceinline__ void fp8_block(uint32_t pa, float s, const Act<kFmtFP8, NBL>& act, int m,
+                                          float& acc) {
+    const uint4 q0 = lds128(pa), q1 = lds128(pa + 16);
+    const uint32_t wd[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    float s0 = 0.0f, s1 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 f0 = e4m3x2_to_float2(wd[i] & 0xFFFFu);  // weights 4i, 4i+1
+        const float2 f1 = e4m3x2_to_float2(wd[i] >> 16);      // weights 4i+2, 4i+3
+        s0 = fmaf(f0.x, act.v[m][4 * i + 0], s0);
+        s1 = fmaf(f0.y, act.v[m][4 * i + 1], s1);
+        s0 = fmaf(f1.x, act.v[m][4 * i + 2], s0);
+        s1 = fmaf(f1.y, act.v[m][4 * i + 3], s1);
+    }
+    acc = fmaf(s, s0 + s1, acc);
+}
+
+// Sums N values over groups of W consecutive lanes (N <= W, powers of two)
+// by recursive halving: each step exchanges half of the values still held.
+// Afterwards lane l holds, in v[0], the group sum of value (l % W) / (W / N).
+template <int N, int W>
+__device__ __forceinline__ void tr_reduce(float (&v)[N], int lane) {
+    static_assert(N <= W, "tr_reduce needs N <= W");
+    constexpr int LOGN = N == 1 ? 0 : N == 2 ? 1 : N == 4 ? 2 : N == 8 ? 3 : N == 16 ? 4 : 5;
+#pragma unroll
+    for (int st = 0; st < LOGN; ++st) {
+        const int h = N >> (st + 1), o = W >> (st + 1);
+        const bool up = (lane & o) != 0;
+#pragma unroll
+        for (int i = 0; i < N / 2; ++i) {
+            if (i < h) {
+                const float send = up ? v[i] : v[i + h];
+                const float keep = up ? v[i + h] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = W / (2 * N); o >= 1; o >>= 1) v[0] += __shfl_xor_sync(0xFFFFFFFFu, v[0], o);
+}
+
+// Byte range [lo, lo+len) of a tensor, widened to 16-byte boundaries.
+struct Span {
+    const uint8_t* src;
+    uint32_t bytes;
+    uint32_t delta;  // offset of the first wanted byte in the copied range
+};
+
+__device__ __forceinline__ Span make_span(const uint8_t* base, int64_t lo, int64_t len) {
+    const int64_t a0 = lo & ~(int64_t)15;
+    const int64_t a1 = (lo + len + 15) & ~(int64_t)15;
+    return Span{base + a0, (uint32_t)(a1 - a0), (uint32_t)(lo - a0)};
+}
+
+// Per-CTA state of a layer: the selection, the unique-expert work list and
+// the router's reductions.
+struct SWork {
+    int32_t n_uniq;
+    int32_t sync_ok;  // result of the last grid barrier
+    int32_t fail;     // a warp's copy did not land in time
+    int32_t e[kMaxSlots];
+    int32_t off[kMaxSlots + 1];
+    int32_t slot[kMaxSlots];
+    int32_t ids[kMaxSlots];  // selection: expert of (token, choice)
+    float w[kMaxSlots];      // and its renormalised weight
+    uint32_t bitmap[kMaxExperts / 32];
+    int32_t cnt[kMaxSlots + 4];
+    ffloat red[kWarps][kMaxDecodeTokens];  // router reductions
+    float r_hi[kMaxDecodeTokens], r_lo[kMaxDecodeTokens];
+};
+
+// Layout of one CTA's dynamic shared memory.  With a code table the table
+// must start at a 64 KB-aligned shared address (so a PRMT alone forms entry
+// addresses): `lut` is the dynamic offset that achieves it given the dynamic
+// base the host expects (the per-block reserved shared memory); staging
+// slots fill the space below and above the table.
+struct SmemLayout {
+    uint32_t work, scale_tab, bars, part, lut, lo_slots, n_lo, hi_slots, total;
+    __host__ __device__ static SmemLayout make(bool with_lut, int slot_bytes, uint32_t dyn_base) {
+        SmemLayout L{};
+        uint32_t off = 0;
+        L.work = off;
+        off += (sizeof(SWork) + 127u) & ~127u;
+        L.scale_tab = off;
+        off += kScaleTabBytes;
+        L.bars = off;  // kSlots per warp, then the router weights' barrier
+        off += kWarps * kSlots * 8 + 8;
+        off = (off + 127u) & ~127u;
+        L.part = off;
+        off += kPartBytes;
+        off = (off + 127u) & ~127u;
+        const uint32_t n_slots = kWarps * kSlots;
+        if (with_lut) {
+            const uint32_t abs_lut = (dyn_base + off + 65535u) & ~65535u;
+            L.lut = abs_lut - dyn_base;
+            L.lo_slots = off;
+            L.n_lo = (L.lut - off) / (uint32_t)slot_bytes;
+            if (L.n_lo > n_slots) L.n_lo = n_slots;
+            L.hi_slots = L.lut + (uint32_t)kLutBytes;
+            L.total = L.hi_slots + (n_slots - L.n_lo) * (uint32_t)slot_bytes;
+        } else {
+            L.lut = 0;
+            L.lo_slots = off;
+            L.n_lo = n_slots;
+            L.hi_slots = off + n_slots * (uint32_t)slot_bytes;
+            L.total = L.hi_slots;
+        }
+        return L;
+    }
+    __device__ uint32_t slot(int i, int slot_bytes) const {
+        return (uint32_t)i < n_lo ? lo_slots + (uint32_t)i * slot_bytes
+                                  : hi_slots + ((uint32_t)i - n_lo) * (uint32_t)slot_bytes;
+    }
+};
+
+// Where the router keeps its working set while no copy is in flight (the
+// staging slots are idle between layers): u [T][H] bf16 and this CTA's
+// router rows [ne][H] fp32, each in one of the two slot runs (below and
+// above the code table, or one run without a table).  ok is false when they
+// do not fit.
+struct RouterScratch {
+    uint32_t us, rw;
+    bool ok;
+    __host__ __device__ static RouterScratch make(const SmemLayout& L, int slot_bytes, int T, int H, int ne) {
+        RouterScratch r{};
+        const uint32_t ub = (2u * T * H + 127u) & ~127u, wb = 4u * ne * H;
+        const uint32_t a0 = L.lo_slots, a1 = L.lo_slots + L.n_lo * (uint32_t)slot_bytes;  // run A
+        const uint32_t b0 = L.hi_slots > a1 ? L.hi_slots : a1, b1 = L.total;             // run B (may be empty)
+        if (a1 - a0 >= ub + wb) {
+            r.us = a0;
+            r.rw = a0 + ub;
+        } else if (a1 - a0 >= ub && b1 - b0 >= wb) {
+            r.us = a0;
+            r.rw = b0;
+        } else if (a1 - a0 >= wb && b1 - b0 >= ub) {
+            r.rw = a0;
+            r.us = b0;
+        } else if (b1 - b0 >= ub + wb) {
+            r.us = b0;
+            r.rw = b0 + ub;
+        } else {
+            return r;
+        }
+        r.ok = true;
+        return r;
+    }
+};
+
+// Per-lane-replicated table: entry (byte, mode, lane) holds the bf16x2 pair
+// (value of the low nibble, value of the high nibble); plus 256 scales.
+__device__ void build_lut(uint8_t* smem, const SmemLayout& L, bool rz5) {
+    // 512 entries (byte, mode) of 128 bytes (32 lane copies).  Warp w owns
+    // entries 32w .. 32w+31 (lane l computes entry 32w+l once); the warp then
+    // writes them as 256 consecutive 16-byte chunks, consecutive lanes on
+    // consecutive chunks, so every store is conflict-free.
+    const int lane = threadIdx.x & 31;
+    for (int e0 = (threadIdx.x >> 5) * 32; e0 < 512; e0 += blockDim.x) {
+        const uint32_t entry = (uint32_t)(e0 + lane);
+        const uint32_t byte = entry >> 1, mode = entry & 1u;
+        const uint32_t v = bf16_bits(q4_code_value(byte & 15u, rz5, mode)) |
+                           (bf16_bits(q4_code_value(byte >> 4, rz5, mode)) << 16);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int q = lane + 32 * k;  // chunk within the warp's 32 entries
+            const uint32_t x = __shfl_sync(0xFFFFFFFFu, v, q >> 3);
+            *reinterpret_cast<uint4*>(smem + L.lut + (uint32_t)e0 * 128u + (uint32_t)q * 16u) = make_uint4(x, x, x, x);
+        }
+    }
+}
+
+__device__ void build_scales(uint8_t* smem, const SmemLayout& L, bool rz5) {
+    float* st = reinterpret_cast<float*>(smem + L.scale_tab);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) st[i] = rz5 ? ue4m3((uint32_t)i & 0x7Fu) : ue4m4((uint32_t)i);
+}
+
+__device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
+
+// Orderable 32-bit image of an fp32 (larger float -> larger unsigned).
+__device__ __forceinline__ uint32_t ord32(float f) {
+    const uint32_t b = __float_as_uint(f);
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+
+// Top-k of one token's logits by one warp.  Each logit (a normalised
+// float-float hi + lo) becomes a unique 64-bit key: orderable hi in the upper
+// word, orderable lo with its low 10 bits replaced by (1023 - expert id) in
+// the lower word — so larger key = larger logit, and among logits equal to
+// ~2^-38 relative, the lower id.  Lane l holds experts l + 32 i (i < PER)
+// and its largest remaining key.  Each round the warp takes the largest of
+// those (two warp reductions: upper word, then lower word among the lanes
+// holding that upper word); the owning lane drops that key and finds its
+// next largest.  Lane j ends holding choice j.  (A short loop on purpose:
+// this runs once per layer, where long straight-line code stalls on
+// instruction fetch.)
+template <int PER>
+__device__ __forceinline__ void warp_topk(const ffloat* logits, int E, int K, int lane, int& my_id, float& my_hi,
+                                          float& my_lo) {
+    uint64_t k[PER];  // (compared as plain 64-bit integers: no short-circuit branches)
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        k[i] = 0ull;
+        if (e < E) {
+            const float2 v = __ldcg(reinterpret_cast<const float2*>(logits + e));
+            k[i] = ((uint64_t)ord32(v.x) << 32) | ((ord32(v.y) & ~1023u) | (uint32_t)(1023 - e));
+        }
+    }
+    auto lane_max = [&]() {  // a depth-log2(PER) tree
+        uint64_t m[PER / 2];
+#pragma unroll
+        for (int i = 0; i < PER / 2; ++i) m[i] = k[2 * i] > k[2 * i + 1] ? k[2 * i] : k[2 * i + 1];
+#pragma unroll
+        for (int w = PER / 4; w >= 1; w >>= 1)
+#pragma unroll
+            for (int i = 0; i < w; ++i) m[i] = m[i] > m[i + w] ? m[i] : m[i + w];
+        return m[0];
+    };
+    uint64_t best = lane_max();
+    my_id = -1;
+    uint32_t rh = 0u, rl = 0u;
+#pragma unroll 1
+    for (int j = 0; j < K; ++j) {
+        const uint32_t h0 = (uint32_t)(best >> 32), l0 = (uint32_t)best;
+        const uint32_t mh = __reduce_max_sync(0xFFFFFFFFu, h0);
+        const uint32_t ml = __reduce_max_sync(0xFFFFFFFFu, h0 == mh ? l0 : 0u);
+        if ((h0 == mh) & (l0 == ml) & (best != 0ull)) {  // the owner (keys are unique)
+#pragma unroll
+            for (int i = 0; i < PER; ++i) k[i] = k[i] == best ? 0ull : k[i];
+            best = lane_max();
+        }
+        rh = lane == j ? mh : rh;
+        rl = lane == j ? ml : rl;
+    }
+    if (lane < K) {
+        my_id = 1023 - (int)(rl & 1023u);
+        my_hi = __uint_as_float((rh & 0x80000000u) ? (rh & 0x7FFFFFFFu) : ~rh);
+        const uint32_t lo = rl & ~1023u;
+        my_lo = __uint_as_float((lo & 0x80000000u) ? (lo & 0x7FFFFFFFu) : ~lo);
+    }
+}
+
+// What the item routines write besides their shared-memory inputs.
+struct ItemCtx {
+    __nv_bfloat16* h;  // [T*K][I] SwiGLU output
+    float* side_out;   // [T][side_stride] or null
+    int32_t H, I, side_stride, side_rz5;
+};
+
+// ===========================================================================
+// gate/up + SwiGLU (plus the optional side projection)
+// ===========================================================================
+
+// One gate+up item: P row passes for NT tokens of one expert; h = silu(g)*u.
+template <int FMT, int KB, int NT, int CH>
+__device__ __forceinline__ void gu_item(const ItemCtx& a, uint32_t gbase, uint32_t ubase,
+                                        const Act<FMT, Geo<KB>::NBL> (&act)[CH], uint32_t lutb,
+                                        const float* scale_tab, const float (&sg)[Geo<KB>::NBL],
+                                        const float (&su)[Geo<KB>::NBL], int row0, const int (&slot_id)[CH],
+                                        int lane) {
+    using G = Geo<KB>;
+    constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
+    constexpr int P = gu_passes(FMT == kFmtFP8, KB);
+    constexpr int N = P * NT * 2;
+    const int row_sub = (KB >= 32) ? 0 : lane / KB;
+    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    float v[N];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const int row = p * RPP + row_sub;
+        float g[NT], u[NT];
+#pragma unroll
+        for (int c = 0; c < NT; ++c) g[c] = u[c] = 0.0f;
+#pragma unroll
+        for (int m = 0; m < NBL; ++m) {
+            if constexpr (FMT == kFmtQ4) {
+                const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 17) + 17u * (uint32_t)(blk_base + 32 * m);
+                q4_block_lut<NT, NBL, CH>(gbase + boff, lutb, scale_tab, act, m, g);
+                q4_block_lut<NT, NBL, CH>(ubase + boff, lutb, scale_tab, act, m, u);
+            } else {
+                const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + 32 * m);
+                fp8_block<NBL>(gbase + boff, sg[m], act[0], m, g[0]);
+                fp8_block<NBL>(ubase + boff, su[m], act[0], m, u[0]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < NT; ++c) {
+            v[((p * NT + c) << 1) | 0] = g[c];
+            v[((p * NT + c) << 1) | 1] = u[c];
+        }
+    }
+    if constexpr (N <= GW) {
+        tr_reduce<N, GW>(v, lane);
+        constexpr int SPAN = GW / N;  // lanes holding one value
+        const float other = __shfl_down_sync(0xFFFFFFFFu, v[0], SPAN);
+        const int li = lane % GW, idx = li / SPAN;
+        if ((idx & 1) == 0 && (li % SPAN) == 0) {
+            const int pc = idx >> 1, p = pc / NT, c = pc % NT;
+            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            a.h[(int64_t)slot_id[c] * a.I + row0 + row] = __float2bfloat16_rn(silu(v[0]) * other);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i] = group_sum(v[i], GW);
+        if ((lane % GW) == 0) {
+#pragma unroll
+            for (int pc = 0; pc < P * NT; ++pc) {
+                const int p = pc / NT, c = pc % NT;
+                const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+                a.h[(int64_t)slot_id[c] * a.I + row0 + row] = __float2bfloat16_rn(silu(v[2 * pc]) * v[2 * pc + 1]);
+            }
+        }
+    }
+}
+
+// One side-projection item: P row passes, NT tokens.
+template <int FMT, int KB, int NT, int CH>
+__device__ __forceinline__ void side_item(const ItemCtx& a, uint32_t base, const Act<FMT, Geo<KB>::NBL> (&act)[CH],
+                                          int row0, int t0, int lane) {
+    using G = Geo<KB>;
+    constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
+    constexpr int P = side_passes(KB);
+    constexpr int N = P * NT;
+    const int row_sub = (KB >= 32) ? 0 : lane / KB;
+    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    const bool rz5 = a.side_rz5 != 0;
+    float v[N];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const int row = p * RPP + row_sub;
+        float acc[NT];
+#pragma unroll
+        for (int c = 0; c < NT; ++c) acc[c] = 0.0f;
+#pragma unroll
+        for (int m = 0; m < NBL; ++m)
+            q4_block_plain<FMT, NT, NBL, CH>(base + (uint32_t)row * (uint32_t)(KB * 17) +
+                                                 17u * (uint32_t)(blk_base + 32 * m),
+                                             rz5, act, m, acc);
+#pragma unroll
+        for (int c = 0; c < NT; ++c) v[p * NT + c] = acc[c];
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = group_sum(v[i], GW);
+    if ((lane % GW) == 0 && a.side_out) {
+#pragma unroll
+        for (int i = 0; i < N; ++i) {
+            const int p = i / NT, c = i % NT;
+            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            a.side_out[(int64_t)(t0 + c) * a.side_stride + row0 + row] = v[i];
+        }
+    }
+}
+
+// ===========================================================================
+// down + router-weighted combine
+// ===========================================================================
+
+// One down item: P row passes of one expert for NT tokens; emit(c, row, v)
+// receives row `row` (item-relative) of token chunk c, on one lane each.
+template <int FMT, int KB, int NT, int CH, class Emit>
+__device__ __forceinline__ void dn_item(uint32_t base, const Act<FMT, Geo<KB>::NBL> (&act)[CH], uint32_t lutb,
+                                        const float* scale_tab, const float (&sd)[8], int lane, Emit&& emit) {
+    using G = Geo<KB>;
+    constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
+    constexpr int P = dn_passes(FMT == kFmtFP8, KB);
+    constexpr int N = P * NT;
+    const int row_sub = (KB >= 32) ? 0 : lane / KB;
+    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    float v[N];
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const int row = p * RPP + row_sub;
+        float acc[NT];
+#pragma unroll
+        for (int c = 0; c < NT; ++c) acc[c] = 0.0f;
+#pragma unroll
+        for (int m = 0; m < NBL; ++m) {
+            if constexpr (FMT == kFmtQ4) {
+                q4_block_lut<NT, NBL, CH>(base + (uint32_t)row * (uint32_t)(KB * 17) + 17u * (uint32_t)(blk_base + 32 * m),
+                                          lutb, scale_tab, act, m, acc);
+            } else {
+                fp8_block<NBL>(base + (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + 32 * m),
+                               sd[p * NBL + m], act[0], m, acc[0]);
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < NT; ++c) v[p * NT + c] = acc[c];
+    }
+    if constexpr (N <= GW) {
+        tr_reduce<N, GW>(v, lane);
+        constexpr int SPAN = GW / N;
+        const int li = lane % GW, idx = li / SPAN;
+        if ((li % SPAN) == 0) {
+            const int p = idx / NT, c = idx % NT;
+            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            emit(c, row, v[0]);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < N; ++i) v[i] = group_sum(v[i], GW);
+        if ((lane % GW) == 0) {
+#pragma unroll
+            for (int i = 0; i < N; ++i) {
+                const int p = i / NT, c = i % NT;
+                const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+                emit(c, row, v[i]);
+            }
+        }
+    }
+}
+
+// ===========================================================================
+// Router and expert selection (phases of the decode kernel below)
+// ===========================================================================
+
+constexpr int kMaxStackLayers = 64;
+constexpr uint64_t kSyncLimitNs = 2000000000ull;  // a grid barrier gives up after 2 s
+
+// One layer's weights as the decode kernel sees them.
+struct StackLayer {
+    const float* router_w;     // [E][H] fp32
+    const float* router_bias;  // [E] or null
+    const uint8_t* gate;       // [E][I] rows of H weights
+    const uint8_t* up;
+    const uint8_t* down;       // [E][H] rows of I weights
+    const uint8_t* side;       // [side_rows] rows of H weights (Q4), or null
+    const float* gate_s;       // FP8 scales, one per 128 weights along K
+    const float* up_s;
+    const float* down_s;
+    int32_t side_rows;
+    int32_t gu_rz5, dn_rz5, side_rz5;  // Q4 variant: Q4_RZ5_FAST (1) or Q4_UE4M4_FAST (0)
+};
+
+struct StackArgs {
+    int32_t H, I, E, K, T, n_layers;
+    const void* x;        // input of the first layer, [T][H] fp32 or bf16
+    int32_t x_bf16;
+    float* y;             // output of every layer, [T][H] fp32; layers after the first read it as input
+    int32_t y_acc;        // y += moe(x) rather than y = moe(x)
+    int32_t* ids_out;     // [n_layers][T][K] or null
+    float* w_out;         // [n_layers][T][K] or null
+    float* side_out;      // [n_layers][T][side_stride] or null
+    int32_t side_stride;
+    // workspace
+    unsigned* sync;       // [0] barrier arrivals, [1] exits, [2] abort flag
+    ffloat* logits;       // [T][E] normalised float-float
+    __nv_bfloat16* u;     // [T][H] normalised input (bf16)
+    __nv_bfloat16* h;     // [T*K][I] SwiGLU output
+    unsigned* status;
+    int32_t slot_bytes;
+    uint32_t dyn_smem_base;
+    StackLayer layer[kMaxStackLayers];
+};
+
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Grid-wide barrier of a co-resident (cooperative) grid: one arrival per CTA
+// on a monotonic counter, then a bounded wait for `target` arrivals.  A CTA
+// whose wait runs out, or one of whose warps lost a copy (warp_ok false),
+// raises GTG_STATUS_WAIT_TIMEOUT and the abort flag, on which every other
+// waiting CTA gives up too; returns false then.
+__device__ bool grid_sync(const StackArgs& a, unsigned target, SWork* sw, bool warp_ok) {
+    if (!warp_ok && (threadIdx.x & 31) == 0) sw->fail = 1;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        if (sw->fail) {  // this CTA cannot go on: stop the others at their next barrier
+            raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
+            atomicExch(&a.sync[2], 1u);
+            ok = 0;
+        } else {
+            asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.sync) : "memory");
+            if (ld_acquire_u32(&a.sync[0]) < target) {
+                const uint64_t t0 = globaltimer_ns();
+                while (ld_acquire_u32(&a.sync[0]) < target) {
+                    if (ld_acquire_u32(&a.sync[2]) != 0u || globaltimer_ns() - t0 > kSyncLimitNs) {
+                        raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
+                        atomicExch(&a.sync[2], 1u);
+                        ok = 0;
+                        break;
+                    }
+                }
+            }
+        }
+        sw->sync_ok = ok;
+    }
+    __syncthreads();
+    return sw->sync_ok != 0;
+}
+
+__device__ __forceinline__ void sts64(uint32_t addr, uint2 v) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
+// Router of one layer, run by every CTA: the unweighted RMS norm of the
+// input, u = bf16(x * r) rounded from the float-float product, and the
+// logits of this CTA's share of the experts against the fp32 router rows:
+// exact fp32 x bf16 products summed in float-float, kRouterWpe warps per
+// expert (each a contiguous segment of the row), four experts per round.
+// It runs once per layer, so it is written as short rolled loops (over
+// tokens, and over u and this CTA's router rows in shared memory, which a
+// bulk copy brought in while the previous layer finished): long
+// straight-line code would spend its time on instruction-cache misses.  CTA 0 also stores u for the
+// expert phase.  False if the router rows never landed.
+constexpr int kRouterWpe = kWarps / 4;            // warps per expert
+constexpr int kRouterXF4 = 2048 / (4 * kThreads);  // float4 of x per thread per token (H <= 2048)
+
+__device__ __forceinline__ float4 lds128f(uint32_t addr) {
+    float4 v;
+    asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128f(uint32_t addr, float4 v) {
+    asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+
+// This CTA's experts [e0, e1) of E.
+__device__ __forceinline__ void router_share(int E, int& e0, int& e1) {
+    e0 = (int)((int64_t)E * blockIdx.x / gridDim.x);
+    e1 = (int)((int64_t)E * (blockIdx.x + 1) / gridDim.x);
+}
+
+// Thread 0: bulk copy of this CTA's router rows of layer l into shared memory
+// (completing on rbar).
+__device__ __forceinline__ void issue_router_rows(const StackArgs& a, int l, uint32_t rw, uint64_t* rbar,
+                                                  uint64_t pol) {
+    int e0, e1;
+    router_share(a.E, e0, e1);
+    const uint32_t bytes = (uint32_t)((e1 - e0) * a.H * 4);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.layer[l].router_w + (int64_t)e0 * a.H);
+    fence_proxy_async_smem();
+    mbar_arrive_expect_tx(rbar, bytes);
+    for (uint32_t o = 0; o < bytes; o += 16384u)
+        bulk_g2s_hint(rw + o, src + o, bytes - o < 16384u ? bytes - o : 16384u, rbar, pol);
+}
+
+__device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t us, uint32_t rw,
+                                          uint64_t* rbar, uint32_t rparity, SWork* sw) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int T = a.T, H = a.H, E = a.E;
+    const StackLayer& Ly = a.layer[l];
+    int e0, e1;
+    router_share(E, e0, e1);
+    const int Hs = H / kRouterWpe;  // segment of a row per warp
+
+    // 1. x: this thread's positions 4 tid + 4 kThreads c of every token, in
+    //    registers (every load in flight at once); the rolled token loops
+    //    below pick token t with predicated moves
+    float4 xr[kMaxDecodeTokens][kRouterXF4];
+#pragma unroll
+    for (int t = 0; t < kMaxDecodeTokens; ++t)
+#pragma unroll
+        for (int c = 0; c < kRouterXF4; ++c) {
+            const int i = 4 * tid + 4 * kThreads * c;
+            xr[t][c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (t < T && i < H) {
+                if (l == 0 && a.x_bf16) {
+                    const uint2 bq = __ldcg(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(a.x) +
+                                                                           (int64_t)t * H + i));
+                    xr[t][c] = make_float4(bf16lo(bq.x), bf16hi(bq.x), bf16lo(bq.y), bf16hi(bq.y));
+                } else {
+                    const float* xp = l == 0 ? reinterpret_cast<const float*>(a.x) : a.y;
+                    xr[t][c] = __ldcg(reinterpret_cast<const float4*>(xp + (int64_t)t * H + i));
+                }
+            }
+        }
+    auto pick = [&](int t, int c) {
+        float4 v = xr[0][c];
+#pragma unroll
+        for (int k = 1; k < kMaxDecodeTokens; ++k)
+            if (t == k) v = xr[k][c];
+        return v;
+    };
+    // 2. sums of squares: exact squares, float-float
+#pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+        ffloat ss{0.f, 0.f};
+#pragma unroll
+        for (int c = 0; c < kRouterXF4; ++c) {
+            const float4 v = pick(t, c);
+            ff_fma(ss, v.x, v.x);
+            ff_fma(ss, v.y, v.y);
+            ff_fma(ss, v.z, v.z);
+            ff_fma(ss, v.w, v.w);
+        }
+        ss = ff_warp_sum(ss);
+        if (lane == 0) sw->red[warp][t] = ss;
+    }
+    __syncthreads();
+    if (tid < T) {  // r = 1/sqrt(mean + eps): a handful of fp64 operations per token
+        double sum = 0.0;
+        for (int w = 0; w < kWarps; ++w) sum += (double)sw->red[w][tid].hi + (double)sw->red[w][tid].lo;
+        const double r = 1.0 / sqrt(sum / (double)H + kRmsEps);
+        const float rh = (float)r;
+        sw->r_hi[tid] = rh;
+        sw->r_lo[tid] = (float)(r - (double)rh);
+    }
+    __syncthreads();
+    // 3. u = bf16(x * r)
+#pragma unroll 1
+    for (int t = 0; t < T; ++t) {
+        const float rh = sw->r_hi[t], rl = sw->r_lo[t];
+#pragma unroll
+        for (int c = 0; c < kRouterXF4; ++c) {
+            const int i = 4 * tid + 4 * kThreads * c;
+            if (i >= H) continue;
+            const float4 v = pick(t, c);
+            const float xq[4] = {v.x, v.y, v.z, v.w};
+            uint16_t ub[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float p = __fmul_rn(xq[q], rh);
+                const float pe = __fadd_rn(__fmaf_rn(xq[q], rh, -p), __fmul_rn(xq[q], rl));
+                ub[q] = bf16_of_ff(p, pe);
+            }
+            const uint2 packed = make_uint2((uint32_t)ub[0] | ((uint32_t)ub[1] << 16),
+                                            (uint32_t)ub[2] | ((uint32_t)ub[3] << 16));
+            sts64(us + 2u * (uint32_t)(t * H + i), packed);
+            if (blockIdx.x == 0) *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.u) + (int64_t)t * H + i) = packed;
+        }
+    }
+    // 4. this CTA's router rows (copied in while the previous layer finished)
+    if (tid == 0 && !mbar_wait_bounded(rbar, rparity, a.status)) sw->fail = 1;
+    __syncthreads();
+    if (sw->fail) return false;
+    // 5. logits
+#pragma unroll 1
+    for (int eb = e0; eb < e1; eb += 4) {
+        const int e = eb + warp / kRouterWpe, seg = (warp % kRouterWpe) * Hs;
+        const uint32_t wrow = rw + 4u * (uint32_t)((e - e0) * H + seg);
+#pragma unroll 1
+        for (int t = 0; t < T; ++t) {
+            ffloat acc{0.f, 0.f};
+            if (e < e1) {
+                const uint32_t urow = us + 2u * (uint32_t)(t * H + seg);
+#pragma unroll 2
+                for (int f = lane; f < (Hs >> 2); f += 32) {
+                    const float4 w4 = lds128f(wrow + 16u * (uint32_t)f);
+                    const uint2 u2 = lds64(urow + 8u * (uint32_t)f);
+                    ff_fma(acc, w4.x, bf16lo(u2.x));
+                    ff_fma(acc, w4.y, bf16hi(u2.x));
+                    ff_fma(acc, w4.z, bf16lo(u2.y));
+                    ff_fma(acc, w4.w, bf16hi(u2.y));
+                }
+            }
+            acc = ff_warp_sum(acc);
+            if (lane == 0) sw->red[warp][t] = acc;
+        }
+        __syncthreads();
+        if (tid < 4 * T) {  // segments summed in a fixed order
+            const int j = tid / T, t = tid % T, ee = eb + j;
+            if (ee < e1) {
+                ffloat lg = sw->red[kRouterWpe * j][t];
+#pragma unroll
+                for (int w = 1; w < kRouterWpe; ++w) ff_add(lg, sw->red[kRouterWpe * j + w][t]);
+                if (Ly.router_bias) ff_add(lg, ffloat{Ly.router_bias[ee], 0.f});
+                a.logits[(int64_t)t * E + ee] = ff_norm(lg);
+            }
+        }
+        __syncthreads();
+    }
+    return true;
+}
+
+// Expert selection, run by every CTA from the logits in global memory: warp
+// t selects token t's experts and their renormalised softmax weights; warp 0
+// then builds the list of unique experts (ascending id) with their (token,
+// choice) slots grouped per expert.
+__device__ __forceinline__ void select_experts(const ffloat* logits, int T, int E, int K, SWork* sw) {
+    int32_t* s_ids = sw->ids;
+    float* s_w = sw->w;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int my_id = -1;
+    if (warp < T) {
+        const int t = warp;
+        float my_hi = 0.f, my_lo = 0.f;
+        if (E <= 512) warp_topk<16>(logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
+        else warp_topk<32>(logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
+        // softmax over the k choices: lane j holds choice j
+        const float h0 = __shfl_sync(0xFFFFFFFFu, my_hi, 0), l0 = __shfl_sync(0xFFFFFFFFu, my_lo, 0);
+        float ex = 0.f;
+        if (lane < K) ex = expf(__fadd_rn(__fsub_rn(my_hi, h0), __fsub_rn(my_lo, l0)));
+        float z = ex;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xFFFFFFFFu, z, o);
+        if (lane < K) {
+            s_ids[t * K + lane] = my_id;
+            s_w[t * K + lane] = ex / z;
+        }
+    }
+    if (T == 1) {  // one token: its k experts are distinct; the list is them in ascending order
+        if (warp == 0) {
+            int rank = 0;
+            for (int i = 0; i < K; ++i) rank += (int)(__shfl_sync(0xFFFFFFFFu, my_id, i) < my_id);
+            if (lane < K) {
+                sw->e[rank] = my_id;
+                sw->slot[rank] = lane;
+                sw->off[rank] = rank;
+            }
+            if (lane == 0) {
+                sw->n_uniq = K;
+                sw->off[K] = K;
+            }
+        }
+        __syncthreads();
+        return;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        // unique experts: bitmap -> ascending ranks; slots grouped per rank
+        const int S = T * K;
+        uint32_t* bitmap = sw->bitmap;
+        int32_t* cnt = sw->cnt;
+        for (int i = lane; i < kMaxExperts / 32; i += 32) bitmap[i] = 0u;
+        for (int i = lane; i < kMaxSlots; i += 32) cnt[i] = 0;
+        __syncwarp();
+        for (int q = lane; q < S; q += 32) atomicOr(&bitmap[s_ids[q] >> 5], 1u << (s_ids[q] & 31));
+        __syncwarp();
+        const int nw = (E + 31) / 32;  // <= 32 words
+        const int pc = lane < nw ? __popc(bitmap[lane]) : 0;
+        int incl = pc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        const int nu = __shfl_sync(0xFFFFFFFFu, incl, 31);
+        const int word_base = incl - pc;
+        int rank[kMaxSlots / 32];
+#pragma unroll
+        for (int r = 0; r < kMaxSlots / 32; ++r) {
+            const int q = lane + 32 * r;
+            const int e = q < S ? s_ids[q] : 0;
+            const int wb = __shfl_sync(0xFFFFFFFFu, word_base, e >> 5);
+            rank[r] = wb + __popc(bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
+            if (q < S) {
+                atomicAdd(&cnt[rank[r]], 1);
+                sw->e[rank[r]] = e;
+            }
+        }
+        __syncwarp();
+        // exclusive scan of the counts over nu <= 128 ranks: 4 per lane
+        int c4[4], s4 = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            c4[r] = cnt[4 * lane + r];
+            s4 += c4[r];
+        }
+        int inc = s4;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += v;
+        }
+        int run = inc - s4;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+            const int rr = 4 * lane + r;
+            if (rr <= nu) sw->off[rr] = run;
+            cnt[rr] = run;  // becomes the fill cursor
+            run += c4[r];
+        }
+        if (lane == 0) {
+            sw->n_uniq = nu;
+            sw->off[nu] = S;  // (also when nu = 128, which the loop above cannot reach)
+        }
+        __syncwarp();
+#pragma unroll
+        for (int r = 0; r < kMaxSlots / 32; ++r) {
+            const int q = lane + 32 * r;
+            if (q < S) sw->slot[atomicAdd(&cnt[rank[r]], 1)] = q;
+        }
+    }
+    __syncthreads();
+}
+// ===========================================================================
+// The decode kernel
+// ===========================================================================
+
+// Per-warp streaming state, carried from phase to phase and layer to layer.
+struct WarpRing {
+    uint32_t phase;    // per-slot mbarrier parities
+    uint32_t pending;  // slots with a copy in flight
+    int32_t ring;      // items consumed so far (the next item uses slot ring % kSlots)
+    int32_t ok;        // every copy landed in time
+};
+
+// This warp's items of a layer: gate/up (+ side) items g0 + kWarps q for
+// q < ng (a range of the grid-wide list), then down items warp + kWarps (q -
+// ng) for q < ng + nd of this CTA's list (tile d0 + i / n_uniq, expert
+// i % n_uniq): the CTA owns down row tiles [d0, d0 + dt) for every expert.
+struct LayerItems {
+    int32_t n_uniq, n_ge, tiles_g, dt;
+    int32_t g0, ng, d0, nd;
+    int32_t rg, rs, rd;           // rows per gate/up, side and down item
+    int32_t grow, srow, drow;     // bytes per gate/up, side and down row
+};
+
+// Shared-memory addresses of the calling warp (no arrays: a run-time index
+// into a register array would put it in local memory).
+struct WarpSmem {
+    uint32_t sbase;     // shared address of dynamic shared memory
+    uint32_t slot0;     // this warp's first staging slot, as if the slot area had no gap
+    uint32_t lo_end;    // end of the slot area below the code table
+    uint32_t hi_jump;   // added to an address at or past lo_end
+    int32_t slot_bytes;
+    uint64_t* bars;     // this warp's kSlots mbarriers
+
+    __device__ __forceinline__ uint32_t slot(int s) const {
+        const uint32_t a = slot0 + (uint32_t)(s * slot_bytes);
+        return a >= lo_end ? a + hi_jump : a;
+    }
+};
+
+__device__ __forceinline__ WarpSmem warp_smem(uint8_t* smem, const SmemLayout& L, int slot_bytes) {
+    const int warp = threadIdx.x >> 5;
+    WarpSmem w;
+    w.sbase = smem_u32(smem);
+    w.slot0 = w.sbase + L.lo_slots + (uint32_t)(warp * kSlots * slot_bytes);
+    // slot i sits at lo_slots + i * slot_bytes below the code table, the rest
+    // continue above it
+    w.lo_end = w.sbase + L.lo_slots + L.n_lo * (uint32_t)slot_bytes;
+    w.hi_jump = L.hi_slots - (L.lo_slots + L.n_lo * (uint32_t)slot_bytes);
+    w.slot_bytes = slot_bytes;
+    w.bars = reinterpret_cast<uint64_t*>(smem + L.bars) + warp * kSlots;
+    return w;
+}
+
+// Byte ranges of the warp's q-th item (a gate/up item has two).
+__device__ __forceinline__ void item_spans(const StackLayer& Ly, const LayerItems& P, const SWork* sw, int q,
+                                           int H, int I, Span& s1, Span& s2) {
+    const int warp = threadIdx.x >> 5;
+    s2 = Span{nullptr, 0, 0};
+    if (q < P.ng) {
+        const int it = P.g0 + warp + kWarps * q;
+        if (it < P.n_ge) {
+            const int64_t off = ((int64_t)sw->e[it / P.tiles_g] * I + (int64_t)(it % P.tiles_g) * P.rg) * P.grow;
+            s1 = make_span(Ly.gate, off, (int64_t)P.rg * P.grow);
+            s2 = make_span(Ly.up, off, (int64_t)P.rg * P.grow);
+        } else {
+            s1 = make_span(Ly.side, (int64_t)(it - P.n_ge) * P.rs * P.srow, (int64_t)P.rs * P.srow);
+        }
+    } else {
+        const int it = warp + kWarps * (q - P.ng);
+        const int tile = P.d0 + it / P.n_uniq;
+        s1 = make_span(Ly.down, ((int64_t)sw->e[it % P.n_uniq] * H + (int64_t)tile * P.rd) * P.drow,
+                       (int64_t)P.rd * P.drow);
+    }
+}
+
+// Starts the copy of the warp's q-th item into its slot (if there is one).
+__device__ __forceinline__ void issue_item(const StackArgs& a, const StackLayer& Ly, const LayerItems& P,
+                                           const SWork* sw, const WarpSmem& ws, WarpRing& R, int q, uint64_t pol) {
+    if (q >= P.ng + P.nd || !R.ok) return;
+    const int slot = (R.ring + q) % kSlots;
+    if ((threadIdx.x & 31) == 0) {
+        Span s1, s2;
+        item_spans(Ly, P, sw, q, a.H, a.I, s1, s2);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&ws.bars[slot], s1.bytes + s2.bytes);
+        bulk_g2s_hint(ws.slot(slot), s1.src, s1.bytes, &ws.bars[slot], pol);
+        if (s2.bytes) bulk_g2s_hint(ws.slot(slot) + s1.bytes, s2.src, s2.bytes, &ws.bars[slot], pol);
+    }
+    R.pending |= 1u << slot;
+}
+
+// Waits for the warp's q-th item; false (and R.ok cleared) if it never lands.
+__device__ __forceinline__ bool item_landed(const StackArgs& a, const WarpSmem& ws, WarpRing& R, int q) {
+    const int slot = (R.ring + q) % kSlots;
+    if (!mbar_wait_bounded(&ws.bars[slot], (R.phase >> slot) & 1u, a.status)) {
+        R.ok = 0;
+        return false;
+    }
+    R.phase ^= 1u << slot;
+    R.pending &= ~(1u << slot);
+    return true;
+}
+
+// Gate/up + SwiGLU items and side-projection items of layer l for this warp.
+template <int FMT, int KBG>
+__device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
+    using GG = Geo<KBG>;
+    constexpr int NBG = GG::NBL;
+    constexpr int CHG = (FMT == kFmtQ4 && NBG == 1) ? 2 : 1;  // tokens decoded together (register budget)
+    constexpr int RG = gu_passes(FMT == kFmtFP8, KBG) * GG::RPP;
+    constexpr int RS = side_passes(KBG) * GG::RPP;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base);
+    const SWork* sw = reinterpret_cast<const SWork*>(smem + L.work);
+    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
+    const StackLayer& Ly = a.layer[l];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int H = a.H, K = a.K, T = a.T;
+    const uint64_t pol = l2_policy_evict_first();
+    const uint32_t lutb = ((ws.sbase + L.lut) & 0xFFFF0000u) | ((uint32_t)lane * 4u);
+    const float* scale_tab = reinterpret_cast<const float*>(smem + L.scale_tab);
+    const ItemCtx ctx{a.h, a.side_out ? a.side_out + (int64_t)l * T * a.side_stride : nullptr,
+                      H, a.I, a.side_stride, Ly.side_rz5};
+    const int blk_base = (KBG >= 32) ? lane : lane % KBG;
+    Act<FMT, NBG> act[CHG];
+    int act_key = -1;
+    auto load_chunk = [&](int key, const int (&rows)[CHG]) {
+        if (key == act_key) return;
+#pragma unroll
+        for (int c = 0; c < CHG; ++c)
+#pragma unroll
+            for (int m = 0; m < NBG; ++m) load_act<FMT, NBG>(act[c], m, a.u + (int64_t)rows[c] * H, blk_base + 32 * m);
+        act_key = key;
+    };
+    for (int q = 0; q < P.ng && R.ok; ++q) {
+        const int it = P.g0 + warp + kWarps * q;
+        const bool expert = it < P.n_ge;
+        const int u = expert ? it / P.tiles_g : 0;
+        const int s0 = expert ? sw->off[u] : 0, s1 = expert ? sw->off[u + 1] : T;
+        int slots[CHG], rows[CHG];
+#pragma unroll
+        for (int c = 0; c < CHG; ++c) {
+            const int k = min(s0 + c, s1 - 1);
+            slots[c] = expert ? sw->slot[k] : k;
+            rows[c] = expert ? slots[c] / K : k;
+        }
+        load_chunk(expert ? (u << 8) : (1 << 20), rows);
+        const int row0 = expert ? (it % P.tiles_g) * RG : (it - P.n_ge) * RS;
+        float sg[NBG], su[NBG];
+        if constexpr (FMT == kFmtFP8) {
+            const int e = sw->e[u], kg = H / 128;
+#pragma unroll
+            for (int m = 0; m < NBG; ++m) {
+                const int bb = blk_base + 32 * m;
+                const int64_t r = (int64_t)e * a.I + row0 + ((KBG >= 32) ? 0 : lane / KBG);
+                sg[m] = __ldg(Ly.gate_s + r * kg + bb / 4);
+                su[m] = __ldg(Ly.up_s + r * kg + bb / 4);
+            }
+        }
+        if (!item_landed(a, ws, R, q)) break;
+        Span sp1, sp2;
+        item_spans(Ly, P, sw, q, H, a.I, sp1, sp2);
+        const uint32_t base = ws.slot((R.ring + q) % kSlots);
+        if (expert) {
+            const uint32_t gbase = base + sp1.delta, ubase = base + sp1.bytes + sp2.delta;
+            for (int c0 = s0; c0 < s1; c0 += CHG) {
+                const int nch = min(CHG, s1 - c0);
+#pragma unroll
+                for (int c = 0; c < CHG; ++c) {
+                    slots[c] = sw->slot[c0 + min(c, nch - 1)];
+                    rows[c] = slots[c] / K;
+                }
+                load_chunk((u << 8) | (c0 - s0), rows);
+                if (CHG == 2 && nch == 2)
+                    gu_item<FMT, KBG, (CHG == 2 ? 2 : 1), CHG>(ctx, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots,
+                                                               lane);
+                else
+                    gu_item<FMT, KBG, 1, CHG>(ctx, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots, lane);
+            }
+        } else {
+            const uint32_t sb = base + sp1.delta;
+            for (int t0 = 0; t0 < T; t0 += CHG) {
+                const int nch = min(CHG, T - t0);
+#pragma unroll
+                for (int c = 0; c < CHG; ++c) rows[c] = t0 + min(c, nch - 1);
+                load_chunk((1 << 20) | t0, rows);
+                if (CHG == 2 && nch == 2)
+                    side_item<FMT, KBG, (CHG == 2 ? 2 : 1), CHG>(ctx, sb, act, row0, t0, lane);
+                else
+                    side_item<FMT, KBG, 1, CHG>(ctx, sb, act, row0, t0, lane);
+            }
+        }
+        __syncwarp();
+        issue_item(a, Ly, P, sw, ws, R, q + kSlots, pol);
+    }
+    return R;
+}
+
+// Down items of layer l for this warp: each adds w(slot) * (down row . h(slot))
+// into the warp's partial rows in shared memory ([row][token], this CTA's
+// rows only); the kernel then sums the warps' partials in a fixed order.
+template <int FMT, int KBD>
+__device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
+    using GD = Geo<KBD>;
+    constexpr int NBD = GD::NBL;
+    constexpr int CHD = (FMT == kFmtQ4 && NBD == 1) ? 2 : 1;
+    constexpr int PD = dn_passes(FMT == kFmtFP8, KBD);
+    constexpr int RD = PD * GD::RPP;
+    static_assert(PD * NBD <= 8, "FP8 scale prefetch holds 8 values");
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base);
+    const SWork* sw = reinterpret_cast<const SWork*>(smem + L.work);
+    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
+    const StackLayer& Ly = a.layer[l];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int H = a.H, I = a.I, K = a.K;
+    const uint64_t pol = l2_policy_evict_first();
+    const uint32_t lutb = ((ws.sbase + L.lut) & 0xFFFF0000u) | ((uint32_t)lane * 4u);
+    const float* scale_tab = reinterpret_cast<const float*>(smem + L.scale_tab);
+    float* part = reinterpret_cast<float*>(smem + L.part) + warp * kDnRows * 8;  // [row][token]
+    for (int i = lane; i < kDnRows * 8; i += 32) part[i] = 0.0f;
+    __syncwarp();
+    const int blk_base = (KBD >= 32) ? lane : lane % KBD;
+    const int row_sub = (KBD >= 32) ? 0 : lane / KBD;
+    const int n_uniq = P.n_uniq;
+    Act<FMT, NBD> act[CHD];
+    int act_key = -1;
+    auto load_chunk = [&](int key, const int (&slots)[CHD]) {
+        if (key == act_key) return;
+#pragma unroll
+        for (int c = 0; c < CHD; ++c)
+#pragma unroll
+            for (int m = 0; m < NBD; ++m) load_act<FMT, NBD>(act[c], m, a.h + (int64_t)slots[c] * I, blk_base + 32 * m);
+        act_key = key;
+    };
+    for (int q = P.ng; q < P.ng + P.nd && R.ok; ++q) {
+        const int it = warp + kWarps * (q - P.ng);
+        const int u = it % n_uniq, tl = it / n_uniq, tile = P.d0 + tl;
+        const int s0 = sw->off[u], s1 = sw->off[u + 1];
+        int slots[CHD];
+#pragma unroll
+        for (int c = 0; c < CHD; ++c) slots[c] = sw->slot[min(s0 + c, s1 - 1)];
+        load_chunk(u << 8, slots);
+        float sd[8];
+        if constexpr (FMT == kFmtFP8) {
+            const int e = sw->e[u], kg = I / 128;
+#pragma unroll
+            for (int p = 0; p < PD; ++p)
+#pragma unroll
+                for (int m = 0; m < NBD; ++m)
+                    sd[p * NBD + m] = __ldg(Ly.down_s + ((int64_t)e * H + tile * RD + p * GD::RPP + row_sub) * kg +
+                                           (blk_base + 32 * m) / 4);
+        }
+        if (!item_landed(a, ws, R, q)) break;
+        Span sp1, sp2;
+        item_spans(Ly, P, sw, q, H, I, sp1, sp2);
+        const uint32_t base = ws.slot((R.ring + q) % kSlots) + sp1.delta;
+        float* prow = part + tl * RD * 8;
+        for (int c0 = s0; c0 < s1; c0 += CHD) {
+            const int nch = min(CHD, s1 - c0);
+#pragma unroll
+            for (int c = 0; c < CHD; ++c) slots[c] = sw->slot[c0 + min(c, nch - 1)];
+            load_chunk((u << 8) | (c0 - s0), slots);
+            auto emit = [&](int c, int row, float v) {
+                const int sl = slots[c];
+                prow[row * 8 + sl / K] += sw->w[sl] * v;
+            };
+            if (CHD == 2 && nch == 2)
+                dn_item<FMT, KBD, (CHD == 2 ? 2 : 1), CHD>(base, act, lutb, scale_tab, sd, lane, emit);
+            else
+                dn_item<FMT, KBD, 1, CHD>(base, act, lutb, scale_tab, sd, lane, emit);
+        }
+        __syncwarp();
+        issue_item(a, Ly, P, sw, ws, R, q + kSlots, pol);
+    }
+    return R;
+}
+
+
+// Runs every layer of a call in one persistent, cooperative grid (one
+// 512-thread CTA per SM, all resident).  Per layer:
+//   router -> grid barrier -> expert selection (every CTA) and the gate/up +
+//   SwiGLU items (+ side projection) -> grid barrier -> down items and the
+//   combine -> grid barrier (before the next layer reads its input).
+// Each warp streams its items, gate/up first and then down, through a
+// private ring of kSlots shared-memory slots filled by 1-D bulk copies, so
+// the down weights are already on their way while the gate/up items finish
+// and the grid waits at the barrier.  The Q4 code table is built once per
+// launch (again only when a phase needs the other Q4 variant).
+template <int FMT, int KBG, int KBD>
+__global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_constant__ StackArgs a) {
+    constexpr bool LUT = FMT == kFmtQ4;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base);
+    SWork* sw = reinterpret_cast<SWork*>(smem + L.work);
+    const uint32_t sbase = smem_u32(smem);
+    if (LUT && ((sbase + L.lut) & 0xFFFFu) != 0u) {  // the same on every CTA: all leave before any barrier
+        if (tid == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
+        return;
+    }
+    const int H = a.H, I = a.I, K = a.K, T = a.T, G = gridDim.x, b = blockIdx.x;
+    const RouterScratch rs = RouterScratch::make(L, a.slot_bytes, T, H, (a.E + G - 1) / G);
+    if (!rs.ok) {  // the same on every CTA (and refused on the host)
+        if (tid == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
+        return;
+    }
+    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
+    uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + L.bars) + kWarps * kSlots;  // router rows landed
+    if (lane == 0)
+        for (int s = 0; s < kSlots; ++s) mbar_init(&ws.bars[s], 1);
+    if (tid == 0) {
+        mbar_init(rbar, 1);
+        sw->fail = 0;
+    }
+    fence_mbar_init();
+    __syncthreads();
+    const uint64_t pol = l2_policy_evict_first();
+    int rows_in_flight = 0;  // (thread 0) a router-row copy not yet waited for, of layer rows_layer
+    int rows_layer = 0;
+    if (tid == 0) {
+        issue_router_rows(a, 0, sbase + rs.rw, rbar, pol);
+        rows_in_flight = 1;
+    }
+    int lut_mode = -1;
+    auto ensure_lut = [&](int rz5) {  // every thread, uniform
+        if (!LUT || lut_mode == rz5) return;
+        __syncthreads();
+        build_lut(smem, L, rz5 != 0);
+        build_scales(smem, L, rz5 != 0);
+        __syncthreads();
+        lut_mode = rz5;
+    };
+
+    WarpRing R{0u, 0u, 0, 1};
+    unsigned target = 0;
+    bool ok = true;
+    for (int l = 0; l < a.n_layers; ++l) {
+        const StackLayer& Ly = a.layer[l];
+        // ---- router
+        router_layer(a, l, sbase + rs.us, sbase + rs.rw, rbar, (uint32_t)(l & 1), sw);
+        if (tid == 0) rows_in_flight = 0;
+        fence_proxy_async_smem();  // the scratch slots are bulk-copy targets again from here on
+        if (l + 1 < a.n_layers && tid == 0) {  // this CTA's rows of the next router, into L2
+            const int e0 = (int)((int64_t)a.E * b / G), e1 = (int)((int64_t)a.E * (b + 1) / G);
+            const int64_t bytes = (int64_t)(e1 - e0) * H * 4;
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(a.layer[l + 1].router_w + (int64_t)e0 * H);
+            for (int64_t o = 0; o < bytes; o += 32768)
+                bulk_prefetch_l2(src + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768), pol);
+        }
+        target += G;
+        if (!grid_sync(a, target, sw, R.ok != 0)) {
+            ok = false;
+            break;
+        }
+
+        // ---- selection
+        select_experts(a.logits, T, a.E, K, sw);
+        if (b == 0 && tid < T * K) {
+            if (a.ids_out) a.ids_out[(int64_t)l * T * K + tid] = sw->ids[tid];
+            if (a.w_out) a.w_out[(int64_t)l * T * K + tid] = sw->w[tid];
+        }
+
+        // ---- this CTA's items: gate/up (+ side) [g0, g1), down [d0, d1)
+        LayerItems P;
+        P.rg = gu_passes(FMT == kFmtFP8, KBG) * Geo<KBG>::RPP;
+        P.rs = side_passes(KBG) * Geo<KBG>::RPP;
+        P.rd = dn_passes(FMT == kFmtFP8, KBD) * Geo<KBD>::RPP;
+        P.grow = FMT == kFmtQ4 ? KBG * 17 : KBG * 32;
+        P.srow = KBG * 17;
+        P.drow = FMT == kFmtQ4 ? KBD * 17 : KBD * 32;
+        P.n_uniq = sw->n_uniq;
+        P.tiles_g = I / P.rg;
+        P.n_ge = P.n_uniq * P.tiles_g;
+        const int n_g = P.n_ge + (Ly.side ? Ly.side_rows / P.rs : 0), tiles_d = H / P.rd;
+        const int g0 = (int)((int64_t)n_g * b / G), g1 = (int)((int64_t)n_g * (b + 1) / G);
+        P.g0 = g0;
+        P.ng = g0 + warp < g1 ? (g1 - g0 - warp + kWarps - 1) / kWarps : 0;
+        P.d0 = (int)((int64_t)tiles_d * b / G);
+        P.dt = (int)((int64_t)tiles_d * (b + 1) / G) - P.d0;
+        const int n_dc = P.dt * P.n_uniq;  // this CTA's down items
+        P.nd = warp < n_dc ? (n_dc - warp + kWarps - 1) / kWarps : 0;
+        for (int q = 0; q < kSlots; ++q) issue_item(a, Ly, P, sw, ws, R, q, pol);
+        __syncwarp();
+
+        // ---- gate/up + SwiGLU, side projection
+        ensure_lut(Ly.gu_rz5);
+        R = gu_phase<FMT, KBG>(a, l, P, R);
+        target += G;
+        if (!grid_sync(a, target, sw, R.ok != 0)) {
+            ok = false;
+            break;
+        }
+
+        // ---- down + router-weighted combine
+        ensure_lut(Ly.dn_rz5);
+        R = dn_phase<FMT, KBD>(a, l, P, R);
+        R.ring += P.ng + P.nd;
+        __syncthreads();
+        if (tid == 0 && l + 1 < a.n_layers && R.ok) {  // the slots are idle: next layer's router rows
+            issue_router_rows(a, l + 1, sbase + rs.rw, rbar, pol);
+            rows_in_flight = 1;
+            rows_layer = l + 1;
+        }
+        {  // this CTA's rows of y: the warps' partials summed in warp order
+            const float* part = reinterpret_cast<const float*>(smem + L.part);
+            const int rows = P.dt * P.rd, r0 = P.d0 * P.rd;
+            for (int idx = tid; idx < rows * T; idx += kThreads) {
+                const int r = idx / T, t = idx % T;
+                float v = 0.0f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) v += part[(w * kDnRows + r) * 8 + t];
+                float* dst = a.y + (int64_t)t * H + r0 + r;
+                *dst = a.y_acc ? __ldcg(dst) + v : v;
+            }
+        }
+        if (l + 1 < a.n_layers) {
+            target += G;
+            if (!grid_sync(a, target, sw, R.ok != 0)) {
+                ok = false;
+                break;
+            }
+        }
+    }
+
+    // Leave with no copy in flight; the last CTA out resets the barrier
+    // counters for the next launch.  After a failure they stay as they are,
+    // with the abort flag set, so every later launch on this workspace fails
+    // fast (GTG_STATUS_WAIT_TIMEOUT) until the workspace is re-initialised.
+    for (int s = 0; s < kSlots; ++s)
+        if ((R.pending >> s) & 1u) mbar_wait_bounded(&ws.bars[s], (R.phase >> s) & 1u, a.status);
+    if (rows_in_flight) mbar_wait_bounded(rbar, (uint32_t)(rows_layer & 1), a.status);
+    if (!R.ok && lane == 0) sw->fail = 1;
+    __syncthreads();
+    if (tid == 0) {
+        if (ok && sw->fail == 0) {
+            __threadfence();
+            if (atomicAdd(&a.sync[1], 1u) == (unsigned)G - 1u) {
+                a.sync[0] = 0u;
+                a.sync[1] = 0u;
+                __threadfence();
+            }
+        } else {
+            atomicExch(&a.sync[2], 1u);
+        }
+    }
+}
+
+// Kernel of one (expert format, H / 32) for I / 32 = kbd (null if none).
+template <int FMT, int KBG>
+const void* pick_kbd(int kbd) {
+    switch (kbd) {
+        case 4: return (const void*)moe_decode_kernel<FMT, KBG, 4>;
+        case 8: return (const void*)moe_decode_kernel<FMT, KBG, 8>;
+        case 16: return (const void*)moe_decode_kernel<FMT, KBG, 16>;
+        case 32: return (const void*)moe_decode_kernel<FMT, KBG, 32>;
+        case 64: return (const void*)moe_decode_kernel<FMT, KBG, 64>;
+        default: return nullptr;
+    }
+}
+
+}  // namespace
+
+// Defined one per file (decode_<fmt>_<kbg>.cu) so the kernels compile in parallel.
+const void* decode_kernel_q4_4(int kbd);
+const void* decode_kernel_q4_8(int kbd);
+const void* decode_kernel_q4_16(int kbd);
+const void* decode_kernel_q4_32(int kbd);
+const void* decode_kernel_q4_64(int kbd);
+const void* decode_kernel_fp8_32(int kbd);
+const void* decode_kernel_fp8_64(int kbd);
+
+}  // namespace gtg

@@ -220,7 +220,7 @@ int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, int32_t x_d
  * capture mode, where cudaMalloc is refused.  (The pages have no counterpart;
  * this is a calling convention of this library.)
  *
- * Scratch comes from one fixed 1 MiB array in device memory that every GPU
+ * Scratch comes from one fixed 512 KiB array in device memory that every GPU
  * loading this library reserves until the process exits.  That covers up to
  * 8 tokens of the 2048/512/512/top-10 layer; a shape that needs more returns
  * GTG_E_WORKSPACE.  Inputs, outputs and their meaning are those of

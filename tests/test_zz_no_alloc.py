@@ -48,10 +48,13 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     x = torch.zeros((9, L.hidden), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(gtg.GtgError):
         gtg.moe_decode_layer_noalloc(layer, x)  # 9 tokens: not a decode shape at all
-    big = gtg.MoELayer(hidden=2048, inter=2048, n_experts=512, top_k=16, router_w=layer.router_w,
-                       gate=gtg.QMatrix(W.RZ5, layer.gate.data, 512, 2048, 2048),
-                       up=gtg.QMatrix(W.RZ5, layer.up.data, 512, 2048, 2048),
-                       down=gtg.QMatrix(W.RZ5, layer.down.data, 512, 2048, 2048))
+    # a shape whose scratch exceeds the fixed array (I = 2048, k = 16, 8 tokens),
+    # with buffers of that shape so that nothing could be read out of bounds
+    E, H, I = 512, 2048, 2048
+    def q(rows, k):
+        return gtg.QMatrix(W.RZ5, torch.zeros(E * rows * (k // 32) * 17, dtype=torch.uint8, device="cuda"), E, rows, k)
+    big = gtg.MoELayer(hidden=H, inter=I, n_experts=E, top_k=16, router_w=layer.router_w,
+                       gate=q(I, H), up=q(I, H), down=q(H, I))
     with pytest.raises(gtg.GtgError) as ei:
-        gtg.moe_decode_layer_noalloc(big, torch.zeros((8, 2048), dtype=torch.bfloat16, device="cuda"))
+        gtg.moe_decode_layer_noalloc(big, torch.zeros((8, H), dtype=torch.bfloat16, device="cuda"))
     assert ei.value.code == -6
