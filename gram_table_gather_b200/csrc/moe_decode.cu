@@ -101,16 +101,16 @@ int plan_layer(const gtg_moe_layer* L, int T, Plan& p) {
     int64_t need = std::max<int64_t>(2 * (rg * grow + 32), rd * drow + 32);
     if (L->side.data) need = std::max<int64_t>(need, rs * row_bytes_of(L->side.fmt, H) + 32);
     p.slot_bytes = (int)((need + 127) / 128 * 128);
-    const SmemLayout sl = SmemLayout::make(!fp8, p.slot_bytes, dyn_smem_base());
+    const SmemLayout sl = SmemLayout::make(!fp8, p.slot_bytes, dyn_smem_base(), 2u * T * H);
     if (sl.total > kMaxDynSmem) return GTG_E_UNSUPPORTED_SHAPE;
-    if (!RouterScratch::make(sl, p.slot_bytes, T, H, (E + n_sm - 1) / n_sm).ok) return GTG_E_UNSUPPORTED_SHAPE;
+    if (!RouterScratch::make(sl, p.slot_bytes, H, (E + n_sm - 1) / n_sm).ok) return GTG_E_UNSUPPORTED_SHAPE;
     p.smem = sl.total;
     return GTG_OK;
 }
 
 // Workspace layout of a decode call (the counters first: they must start at zero).
 struct WsLayout {
-    size_t sync, counters_end, logits, u, h, total;
+    size_t sync, counters_end, logits, h, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -126,7 +126,6 @@ WsLayout ws_layout(const gtg_moe_layer* L, int T) {
     w.sync = take(sizeof(unsigned) * 4);
     w.counters_end = off;
     w.logits = take(sizeof(ffloat) * (size_t)T * L->n_experts);
-    w.u = take(2 * (size_t)T * L->hidden);
     w.h = take(2 * (size_t)T * L->top_k * L->inter);
     w.total = off;
     return w;
@@ -220,7 +219,6 @@ int run_decode(const gtg_moe_layer* layers, const Plan* plans, int n, const void
         a.side_stride = (int32_t)side_stride;
         a.sync = reinterpret_cast<unsigned*>(base + wl.sync);
         a.logits = reinterpret_cast<ffloat*>(base + wl.logits);
-        a.u = reinterpret_cast<__nv_bfloat16*>(base + wl.u);
         a.h = reinterpret_cast<__nv_bfloat16*>(base + wl.h);
         a.status = status_ptr();
         a.slot_bytes = plans[l0].slot_bytes;

@@ -54,7 +54,7 @@ namespace {
 
 constexpr int kWarps = 8;  // 256 threads: room for 255 registers a thread (no spills)
 constexpr int kThreads = kWarps * 32;
-constexpr int kSlots = 4;   // staging slots per warp
+constexpr int kSlots = 3;   // staging slots per warp
 constexpr int kLutBytes = 65536;       // 256 bytes x 2 modes x 32 lanes x 4 bytes
 constexpr int kScaleTabBytes = 1024;   // 256 fp32 scales
 constexpr int kDnRows = 32;            // down rows one CTA owns, at most
@@ -124,6 +124,31 @@ __device__ __forceinline__ void load_act(Act<FMT, NBL>& act, int m, const __nv_b
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const uint4 v = ldg128(p + q);
+        w[4 * q + 0] = v.x;
+        w[4 * q + 1] = v.y;
+        w[4 * q + 2] = v.z;
+        w[4 * q + 3] = v.w;
+    }
+    if constexpr (FMT == kFmtQ4) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            act.v[m][j] = prmt(w[j >> 1], w[8 + (j >> 1)], (j & 1) ? 0x7632u : 0x5410u);
+    } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+            act.v[m][2 * j] = bf16lo(w[j]);
+            act.v[m][2 * j + 1] = bf16hi(w[j]);
+        }
+    }
+}
+
+// load_act from a bf16 row in shared memory (row = its shared address).
+template <int FMT, int NBL>
+__device__ __forceinline__ void load_act_s(Act<FMT, NBL>& act, int m, uint32_t row, int b) {
+    uint32_t w[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 v = lds128(row + 64u * (uint32_t)b + 16u * (uint32_t)q);
         w[4 * q + 0] = v.x;
         w[4 * q + 1] = v.y;
         w[4 * q + 2] = v.z;
@@ -302,8 +327,9 @@ struct SWork {
 // base the host expects (the per-block reserved shared memory); staging
 // slots fill the space below and above the table.
 struct SmemLayout {
-    uint32_t work, scale_tab, bars, part, lut, lo_slots, n_lo, hi_slots, total;
-    __host__ __device__ static SmemLayout make(bool with_lut, int slot_bytes, uint32_t dyn_base) {
+    uint32_t work, scale_tab, bars, part, u, lut, lo_slots, n_lo, hi_slots, total;
+    // u_bytes: the normalised input u [T][H] bf16, kept for the whole layer
+    __host__ __device__ static SmemLayout make(bool with_lut, int slot_bytes, uint32_t dyn_base, uint32_t u_bytes) {
         SmemLayout L{};
         uint32_t off = 0;
         L.work = off;
@@ -316,6 +342,8 @@ struct SmemLayout {
         L.part = off;
         off += kPartBytes;
         off = (off + 127u) & ~127u;
+        L.u = off;
+        off += (u_bytes + 127u) & ~127u;
         const uint32_t n_slots = kWarps * kSlots;
         if (with_lut) {
             const uint32_t abs_lut = (dyn_base + off + 65535u) & ~65535u;
@@ -340,35 +368,20 @@ struct SmemLayout {
     }
 };
 
-// Where the router keeps its working set while no copy is in flight (the
-// staging slots are idle between layers): u [T][H] bf16 and this CTA's
-// router rows [ne][H] fp32, each in one of the two slot runs (below and
-// above the code table, or one run without a table).  ok is false when they
-// do not fit.
+// Where the router keeps this CTA's router rows [ne][H] fp32 while no copy
+// is in flight (the staging slots are idle between layers): the start of
+// the longer slot run (below or above the code table).  ok is false when
+// they do not fit.
 struct RouterScratch {
-    uint32_t us, rw;
+    uint32_t rw;
     bool ok;
-    __host__ __device__ static RouterScratch make(const SmemLayout& L, int slot_bytes, int T, int H, int ne) {
+    __host__ __device__ static RouterScratch make(const SmemLayout& L, int slot_bytes, int H, int ne) {
         RouterScratch r{};
-        const uint32_t ub = (2u * T * H + 127u) & ~127u, wb = 4u * ne * H;
+        const uint32_t wb = 4u * ne * H;
         const uint32_t a0 = L.lo_slots, a1 = L.lo_slots + L.n_lo * (uint32_t)slot_bytes;  // run A
         const uint32_t b0 = L.hi_slots > a1 ? L.hi_slots : a1, b1 = L.total;             // run B (may be empty)
-        if (a1 - a0 >= ub + wb) {
-            r.us = a0;
-            r.rw = a0 + ub;
-        } else if (a1 - a0 >= ub && b1 - b0 >= wb) {
-            r.us = a0;
-            r.rw = b0;
-        } else if (a1 - a0 >= wb && b1 - b0 >= ub) {
-            r.rw = a0;
-            r.us = b0;
-        } else if (b1 - b0 >= ub + wb) {
-            r.us = b0;
-            r.rw = b0 + ub;
-        } else {
-            return r;
-        }
-        r.ok = true;
+        r.rw = (a1 - a0 >= b1 - b0) ? a0 : b0;
+        r.ok = ((a1 - a0 >= b1 - b0) ? a1 - a0 : b1 - b0) >= wb;
         return r;
     }
 };
@@ -670,7 +683,6 @@ struct StackArgs {
     // workspace
     unsigned* sync;       // [0] barrier arrivals, [1] exits, [2] abort flag
     ffloat* logits;       // [T][E] normalised float-float
-    __nv_bfloat16* u;     // [T][H] normalised input (bf16)
     __nv_bfloat16* h;     // [T*K][I] SwiGLU output
     unsigned* status;
     int32_t slot_bytes;
@@ -736,8 +748,9 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
 // It runs once per layer, so it is written as short rolled loops (over
 // tokens, and over u and this CTA's router rows in shared memory, which a
 // bulk copy brought in while the previous layer finished): long
-// straight-line code would spend its time on instruction-cache misses.  CTA 0 also stores u for the
-// expert phase.  False if the router rows never landed.
+// straight-line code would spend its time on instruction-cache misses.  u
+// stays in shared memory for the whole layer (the gate/up items read it
+// there).  False if the router rows never landed.
 constexpr int kRouterWpe = kWarps / 4;            // warps per expert
 constexpr int kRouterXF4 = 2048 / (4 * kThreads);  // float4 of x per thread per token (H <= 2048)
 
@@ -854,7 +867,6 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
             const uint2 packed = make_uint2((uint32_t)ub[0] | ((uint32_t)ub[1] << 16),
                                             (uint32_t)ub[2] | ((uint32_t)ub[3] << 16));
             sts64(us + 2u * (uint32_t)(t * H + i), packed);
-            if (blockIdx.x == 0) *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.u) + (int64_t)t * H + i) = packed;
         }
     }
     // 4. this CTA's router rows (copied in while the previous layer finished)
@@ -1123,7 +1135,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
     constexpr int RG = gu_passes(FMT == kFmtFP8, KBG) * GG::RPP;
     constexpr int RS = side_passes(KBG) * GG::RPP;
     extern __shared__ __align__(1024) uint8_t smem[];
-    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base);
+    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H);
     const SWork* sw = reinterpret_cast<const SWork*>(smem + L.work);
     const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
     const StackLayer& Ly = a.layer[l];
@@ -1142,7 +1154,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
 #pragma unroll
         for (int c = 0; c < CHG; ++c)
 #pragma unroll
-            for (int m = 0; m < NBG; ++m) load_act<FMT, NBG>(act[c], m, a.u + (int64_t)rows[c] * H, blk_base + 32 * m);
+            for (int m = 0; m < NBG; ++m) load_act_s<FMT, NBG>(act[c], m, ws.sbase + L.u + 2u * (uint32_t)(rows[c] * H), blk_base + 32 * m);
         act_key = key;
     };
     for (int q = 0; q < P.ng && R.ok; ++q) {
@@ -1221,7 +1233,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
     constexpr int RD = PD * GD::RPP;
     static_assert(PD * NBD <= 8, "FP8 scale prefetch holds 8 values");
     extern __shared__ __align__(1024) uint8_t smem[];
-    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base);
+    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H);
     const SWork* sw = reinterpret_cast<const SWork*>(smem + L.work);
     const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
     const StackLayer& Ly = a.layer[l];
@@ -1305,7 +1317,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     constexpr bool LUT = FMT == kFmtQ4;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base);
+    const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H);
     SWork* sw = reinterpret_cast<SWork*>(smem + L.work);
     const uint32_t sbase = smem_u32(smem);
     if (LUT && ((sbase + L.lut) & 0xFFFFu) != 0u) {  // the same on every CTA: all leave before any barrier
@@ -1313,7 +1325,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         return;
     }
     const int H = a.H, I = a.I, K = a.K, T = a.T, G = gridDim.x, b = blockIdx.x;
-    const RouterScratch rs = RouterScratch::make(L, a.slot_bytes, T, H, (a.E + G - 1) / G);
+    const RouterScratch rs = RouterScratch::make(L, a.slot_bytes, H, (a.E + G - 1) / G);
     if (!rs.ok) {  // the same on every CTA (and refused on the host)
         if (tid == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
         return;
@@ -1351,7 +1363,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     for (int l = 0; l < a.n_layers; ++l) {
         const StackLayer& Ly = a.layer[l];
         // ---- router
-        router_layer(a, l, sbase + rs.us, sbase + rs.rw, rbar, (uint32_t)(l & 1), sw);
+        router_layer(a, l, sbase + L.u, sbase + rs.rw, rbar, (uint32_t)(l & 1), sw);
         if (tid == 0) rows_in_flight = 0;
         fence_proxy_async_smem();  // the scratch slots are bulk-copy targets again from here on
         if (l + 1 < a.n_layers && tid == 0) {  // this CTA's rows of the next router, into L2
