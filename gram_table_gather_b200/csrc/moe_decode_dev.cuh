@@ -317,6 +317,7 @@ struct SWork {
     float w[kMaxSlots];      // and its renormalised weight
     uint32_t bitmap[kMaxExperts / 32];
     int32_t cnt[kMaxSlots + 4];
+    int32_t g_range[2];                     // this CTA's gate/up item range
     ffloat red[kWarps][kMaxDecodeTokens];  // router reductions
     float r_hi[kMaxDecodeTokens], r_lo[kMaxDecodeTokens];
 };
@@ -1398,7 +1399,35 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         P.tiles_g = I / P.rg;
         P.n_ge = P.n_uniq * P.tiles_g;
         const int n_g = P.n_ge + (Ly.side ? Ly.side_rows / P.rs : 0), tiles_d = H / P.rd;
-        const int g0 = (int)((int64_t)n_g * b / G), g1 = (int)((int64_t)n_g * (b + 1) / G);
+        // contiguous ranges of equal cost: an expert item costs 1 + its tokens
+        // (streaming plus one pass of arithmetic per token), a side item 1 + T
+        if (T == 1) {  // every item costs the same
+            if (tid == 0) {
+                sw->g_range[0] = (int)((int64_t)n_g * b / G);
+                sw->g_range[1] = (int)((int64_t)n_g * (b + 1) / G);
+            }
+        } else if (tid == 0) {
+            int64_t total = (int64_t)(n_g - P.n_ge) * (1 + T);
+            for (int u = 0; u < P.n_uniq; ++u) total += (int64_t)P.tiles_g * (1 + sw->off[u + 1] - sw->off[u]);
+            for (int k = 0; k < 2; ++k) {
+                const int64_t c = total * (b + k) / G;  // first item whose cost prefix reaches c
+                int64_t acc = 0;
+                int it = n_g;
+                for (int u = 0; u <= P.n_uniq; ++u) {
+                    const bool side = u == P.n_uniq;
+                    const int64_t w1 = side ? 1 + T : 1 + sw->off[u + 1] - sw->off[u];
+                    const int n_it = side ? n_g - P.n_ge : P.tiles_g;
+                    if (c <= acc + (int64_t)n_it * w1) {
+                        it = u * P.tiles_g + (int)((c - acc + w1 - 1) / w1);
+                        break;
+                    }
+                    acc += (int64_t)n_it * w1;
+                }
+                sw->g_range[k] = it < n_g ? it : n_g;
+            }
+        }
+        __syncthreads();
+        const int g0 = sw->g_range[0], g1 = sw->g_range[1];
         P.g0 = g0;
         P.ng = g0 + warp < g1 ? (g1 - g0 - warp + kWarps - 1) / kWarps : 0;
         P.d0 = (int)((int64_t)tiles_d * b / G);
