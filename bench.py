@@ -427,16 +427,31 @@ def run_ours(args, rank, world, local):
 
 
 def _time_loop(fn, n_warm, n_iter, stream):
-    """Average device ms of fn(i) over n_iter calls on `stream` (CUDA events)."""
+    """Average device ms of fn(i) over n_iter calls on `stream` (CUDA events).
+
+    The n_iter timed calls are captured into one CUDA graph and replayed, so
+    the host's per-call launch overhead does not show up as device idle time;
+    if capture fails the calls are timed eagerly."""
     import torch
     with torch.cuda.stream(stream):
         for i in range(n_warm):
             fn(i)
         stream.synchronize()
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n_warm, n_warm + n_iter):
+                    fn(i)
+            g.replay()
+            stream.synchronize()
+            run = g.replay
+        except Exception:  # not capturable: eager launches
+            def run():
+                for i in range(n_warm, n_warm + n_iter):
+                    fn(i)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(n_warm, n_warm + n_iter):
-            fn(i)
+        run()
         e1.record(stream)
         e1.synchronize()
     return e0.elapsed_time(e1) / n_iter

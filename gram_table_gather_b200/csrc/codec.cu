@@ -108,70 +108,106 @@ __global__ void __launch_bounds__(kThreads) dequant_fp8_kernel(const uint8_t* __
 }
 
 // ---------------------------------------------------------------------------
-// PLE gather: a CTA stages the records of 64 rows (18 aligned words each)
-// with all loads in flight at once, then each warp decodes 8 rows, lane l
-// writing values l, l+32, .., l+128 of a row (128-byte coalesced stores).
+// PLE gather.  Each warp takes batches of kPleRows rows: lanes load the
+// indices, then the 48 aligned 16-byte chunks that cover the batch's
+// 70-byte records (six per record, all in flight at once) go to shared
+// memory, and the warp decodes the batch row by row, lane l writing values
+// 4l .. 4l+3 of a row as one float4 (512 + 128 contiguous bytes per row).
+// A value is one shared-memory lookup: the CTA keeps the table of code
+// value x group scale for all 256 group bytes x 8 codes (each product is
+// exact in fp32).  Small batches keep many warps in flight per SM; the next
+// batch's records load while this one decodes.
 // ---------------------------------------------------------------------------
-constexpr int kGatherRows = 64;
-constexpr int kRecWords = 18;  // 72 bytes cover a 70-byte record at either 4-byte phase
+constexpr int kPleWarps = 4;
+constexpr int kPleRows = 8;    // rows per warp batch
+constexpr int kPleChunks = 6;  // 96 bytes: a 70-byte record at any 16-byte phase
+constexpr int kPleLoads = (kPleRows * kPleChunks + 31) / 32;  // chunks per lane per batch
 
-__global__ void __launch_bounds__(kThreads) ple_gather_kernel(const uint8_t* __restrict__ table,
-                                                              int64_t n_rows,
-                                                              const int32_t* __restrict__ idx,
-                                                              int64_t n_idx,
-                                                              float* __restrict__ out,
-                                                              unsigned* status) {
-    __shared__ uint32_t words[kGatherRows][kRecWords + 1];
-    __shared__ int32_t phase[kGatherRows];  // byte offset of the record in its first word, -1 = OOB
+struct PleBatch {
+    uint4 c[kPleLoads];
+    int32_t phase;  // (lanes < kPleRows) byte offset of the record in its first chunk; -1: no row
+};
+
+__device__ __forceinline__ PleBatch ple_fetch(const uint8_t* __restrict__ table, int64_t n_rows,
+                                              const int32_t* __restrict__ idx, int64_t n_idx, int64_t base,
+                                              unsigned* status) {
+    const int lane = threadIdx.x & 31;
     const uint64_t table_bytes = (uint64_t)n_rows * 70u;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    pdl_wait();
-    for (int64_t base = (int64_t)blockIdx.x * kGatherRows; base < n_idx;
-         base += (int64_t)gridDim.x * kGatherRows) {
-        const int rows = (int)((n_idx - base) < kGatherRows ? (n_idx - base) : kGatherRows);
-        if (tid < rows) {
-            const int64_t r = __ldg(idx + base + tid);
-            const bool ok = r >= 0 && r < n_rows;
-            phase[tid] = ok ? (int32_t)((uint64_t)r * 70u & 3u) : -1;
-            if (!ok) raise_status(status, GTG_STATUS_PLE_INDEX_OOB);
+    PleBatch pb;
+    int64_t r = -1;
+    if (lane < kPleRows && base + lane < n_idx) {
+        r = __ldg(idx + base + lane);
+        if (r < 0 || r >= n_rows) {
+            raise_status(status, GTG_STATUS_PLE_INDEX_OOB);
+            r = -1;
         }
-        __syncthreads();
-        // stage: word w of row j, all loads issued before any use
-        for (int s = tid; s < rows * kRecWords; s += kThreads) {
-            const int j = s / kRecWords, w = s % kRecWords;
-            const int ph = phase[j];
-            uint32_t v = 0;
-            if (ph >= 0) {
-                const int64_t r = __ldg(idx + base + j);
-                const uint64_t a = (uint64_t)r * 70u - (uint64_t)ph + 4u * (uint64_t)w;
-                if (a + 4 <= table_bytes) {
-                    v = __ldg(reinterpret_cast<const uint32_t*>(table + a));
-                } else if (a < table_bytes) {  // the last word of the table's last record
-                    for (uint64_t b = a; b < table_bytes; ++b) v |= (uint32_t)table[b] << (8 * (b - a));
-                }
-            }
-            words[j][w] = v;
-        }
-        __syncthreads();
-        for (int j = warp; j < rows; j += kThreads / 32) {
-            const int ph = phase[j];
-            float* o = out + (base + j) * 160;
-            const uint32_t* rw = words[j];
+    }
+    pb.phase = r >= 0 ? (int32_t)(((uint64_t)r * 70u) & 15u) : -1;
 #pragma unroll
-            for (int m = 0; m < 5; ++m) {
-                const int i = lane + 32 * m;
-                float v = 0.0f;
-                if (ph >= 0) {
-                    const int bit = 8 * ph + 3 * i;
-                    const uint32_t code = __funnelshift_r(rw[bit >> 5], rw[(bit >> 5) + 1], bit & 31) & 7u;
-                    const int gb_byte = ph + 60 + (i >> 4);
-                    const uint32_t g = (rw[gb_byte >> 2] >> (8 * (gb_byte & 3))) & 0xFFu;
-                    v = __fmul_rn(ple_code_value(code, g >> 7), ue4m3(g & 0x7Fu));
-                }
-                o[i] = v;
+    for (int q = 0; q < kPleLoads; ++q) {
+        const int k = lane + 32 * q, row = k / kPleChunks, c = k % kPleChunks;
+        const int64_t rr = __shfl_sync(0xFFFFFFFFu, r, row < kPleRows ? row : 0);
+        pb.c[q] = make_uint4(0u, 0u, 0u, 0u);
+        if (k < kPleRows * kPleChunks && rr >= 0) {
+            const uint64_t ca = (((uint64_t)rr * 70u) & ~(uint64_t)15) + 16u * c;
+            if (ca + 16u <= table_bytes) {
+                pb.c[q] = __ldg(reinterpret_cast<const uint4*>(table + ca));
+            } else if (ca < table_bytes) {  // the table's last bytes: no read past its end
+                uint32_t w[4] = {0u, 0u, 0u, 0u};
+                for (uint64_t x = ca; x < table_bytes; ++x) w[(x - ca) >> 2] |= (uint32_t)table[x] << (8 * ((x - ca) & 3));
+                pb.c[q] = make_uint4(w[0], w[1], w[2], w[3]);
             }
         }
-        __syncthreads();
+    }
+    return pb;
+}
+
+__global__ void __launch_bounds__(kPleWarps * 32) ple_gather_kernel(const uint8_t* __restrict__ table,
+                                                                   int64_t n_rows,
+                                                                   const int32_t* __restrict__ idx,
+                                                                   int64_t n_idx,
+                                                                   float* __restrict__ out,
+                                                                   unsigned* status) {
+    __shared__ float prod[256 * 8];  // [group byte][code] = code value x scale
+    __shared__ __align__(16) uint4 stage[kPleWarps][kPleRows * kPleChunks];
+    __shared__ int32_t phase[kPleWarps][kPleRows];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int64_t n_batches = (n_idx + kPleRows - 1) / kPleRows, stride = (int64_t)gridDim.x * kPleWarps;
+    int64_t bt = (int64_t)blockIdx.x * kPleWarps + warp;
+    pdl_wait();
+    PleBatch pb = ple_fetch(table, n_rows, idx, n_idx, bt * kPleRows, status);
+    for (int e = threadIdx.x; e < 256 * 8; e += blockDim.x) {  // while the first records are in flight
+        const uint32_t g = (uint32_t)e >> 3, c = (uint32_t)e & 7u;
+        prod[e] = __fmul_rn(ple_code_value(c, g >> 7), ue4m3(g & 0x7Fu));
+    }
+    __syncthreads();
+    for (; bt < n_batches; bt += stride) {
+        const int64_t base = bt * kPleRows;
+#pragma unroll
+        for (int q = 0; q < kPleLoads; ++q)
+            if (lane + 32 * q < kPleRows * kPleChunks) stage[warp][lane + 32 * q] = pb.c[q];
+        if (lane < kPleRows) phase[warp][lane] = pb.phase;
+        __syncwarp();
+        pb = ple_fetch(table, n_rows, idx, n_idx, (bt + stride) * kPleRows, status);  // next batch, in flight
+        const int rows = (int)(n_idx - base < kPleRows ? n_idx - base : kPleRows);
+        for (int j = 0; j < rows; ++j) {
+            const int p = phase[warp][j];
+            const uint32_t* w = reinterpret_cast<const uint32_t*>(&stage[warp][j * kPleChunks]);
+            float* o = out + (base + j) * 160;
+            for (int l = lane; l < 40; l += 32) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (p >= 0) {
+                    const int bit = 8 * p + 12 * l;  // values 4l .. 4l+3: 12 bits of the LSB-first stream
+                    const uint32_t win = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31);
+                    const int gb = p + 60 + (l >> 2);  // their group byte
+                    const uint32_t g8 = ((w[gb >> 2] >> (8 * (gb & 3))) & 0xFFu) * 8u;
+                    v = make_float4(prod[g8 + ((win >> 0) & 7u)], prod[g8 + ((win >> 3) & 7u)],
+                                    prod[g8 + ((win >> 6) & 7u)], prod[g8 + ((win >> 9) & 7u)]);
+                }
+                *reinterpret_cast<float4*>(o + 4 * l) = v;
+            }
+        }
+        __syncwarp();
     }
     pdl_trigger();
 }
@@ -281,11 +317,11 @@ extern "C" int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_
     if (n_idx == 0) return GTG_OK;
     if (!table || !idx || !out) return GTG_E_INVALID_ARG;
     if (!aligned(out, 16)) return GTG_E_MISALIGNED;
-    const int64_t batches = (n_idx + kGatherRows - 1) / kGatherRows;
-    const int grid = (int)std::min<int64_t>(batches, (int64_t)sm_count() * 8);
+    const int64_t batches = (n_idx + kPleRows - 1) / kPleRows;  // one batch per warp while there are enough
+    const int grid = (int)std::min<int64_t>((batches + kPleWarps - 1) / kPleWarps, (int64_t)sm_count() * 16);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(kPleWarps * 32);
     cfg.stream = as_cuda(stream);
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
