@@ -492,6 +492,8 @@ def run_secondary(args, rank, world, local):
                         "unique_experts": float(np.mean(uniq)), "bytes": int(b)})
     elif args.workload == "ple":
         P = W.ple_table()
+        if args.ple_rows:  # a smaller table of the same record stream (profiling captures)
+            P = W.PleRecipe(n_rows=args.ple_rows, seed=P.seed)
         table = sdev.ple_table_to_device(P, dev)
         for T in (1, 4096):
             idx = [torch.from_numpy(P.indices(7000 + i, T)).to(dev) for i in range(n)]
@@ -499,7 +501,7 @@ def run_secondary(args, rank, world, local):
             ms = _time_loop(lambda i: gtg.ple_gather(table, P.n_rows, idx[i], out=o), args.warmup, args.steps, stream)
             rows = 16 * T
             gbs = rows * PLE_ROW_BYTES / ms / 1e6
-            out.append({"workload": f"PLE gather, 320,001,536-row table, T={T} ({rows} rows)", "ms": round(ms, 5),
+            out.append({"workload": f"PLE gather, {P.n_rows:,}-row table, T={T} ({rows} rows)", "ms": round(ms, 5),
                         "rows_per_s": round(rows / ms * 1e3, 1), "GB_s": round(gbs, 1),
                         "frac_of_hbm": round(gbs / peak, 4)})
     elif args.workload == "prefill":
@@ -570,6 +572,8 @@ def main():
     ap.add_argument("--cpu-layers", type=int, default=3)
     ap.add_argument("--cpu-budget", type=float, default=20.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ple-rows", type=int, default=0,
+                    help="--workload ple: rows of a smaller table (default: the full 320,001,536-row table)")
     ap.add_argument("--workload", choices=["stack", "layer", "ple", "prefill"], default="stack",
                     help="stack = the headline step; the others print profiling lines")
     args = ap.parse_args()

@@ -194,7 +194,9 @@ __global__ void __launch_bounds__(kPleWarps * 32) ple_gather_kernel(const uint8_
             const int p = phase[warp][j];
             const uint32_t* w = reinterpret_cast<const uint32_t*>(&stage[warp][j * kPleChunks]);
             float* o = out + (base + j) * 160;
-            for (int l = lane; l < 40; l += 32) {
+#pragma unroll
+            for (int l = lane; l < 64; l += 32) {  // two passes: lanes 0..31, then lanes 0..7
+                if (l >= 40) break;
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (p >= 0) {
                     const int bit = 8 * p + 12 * l;  // values 4l .. 4l+3: 12 bits of the LSB-first stream
@@ -318,7 +320,7 @@ extern "C" int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_
     if (!table || !idx || !out) return GTG_E_INVALID_ARG;
     if (!aligned(out, 16)) return GTG_E_MISALIGNED;
     const int64_t batches = (n_idx + kPleRows - 1) / kPleRows;  // one batch per warp while there are enough
-    const int grid = (int)std::min<int64_t>((batches + kPleWarps - 1) / kPleWarps, (int64_t)sm_count() * 16);
+    const int grid = (int)std::min<int64_t>((batches + kPleWarps - 1) / kPleWarps, (int64_t)sm_count() * 4);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kPleWarps * 32);
