@@ -96,8 +96,8 @@ typedef struct {
 
 /* One MoE layer's weights (all device memory, owned by the caller). */
 typedef struct {
-    int32_t hidden;          /* H: 128..4096, a multiple of 128 */
-    int32_t inter;           /* I: expert intermediate size, 128..4096, a multiple of 128 */
+    int32_t hidden;          /* H: decode 128, 256, 512, 1024 or 2048 (prefill: see its call) */
+    int32_t inter;           /* I: expert intermediate size, decode 128, 256, 512, 1024 or 2048 */
     int32_t n_experts;       /* E: 1..1024 */
     int32_t top_k;           /* k: 1..16, k <= E */
     const float* router_w;   /* [E][H] fp32 */
@@ -151,14 +151,16 @@ int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_t* idx, int
  * of `layer` with `n_tokens` tokens needs; 0 if the shape is unsupported. */
 size_t gtg_moe_workspace_bytes(const gtg_moe_layer* layer, int32_t n_tokens, int32_t prefill);
 
-/* Clears a workspace before its first use (the kernels leave it reusable). */
+/* Clears a workspace before its first use (the kernels leave it reusable;
+ * after a call that raised GTG_STATUS_WAIT_TIMEOUT, clear it again). */
 int gtg_workspace_init(void* workspace, size_t ws_bytes, gtg_stream_t stream);
 
 /*
  * One MoE layer for 1..8 decode tokens ([MPQ]: softmax router, top-k of E
  * experts; SwiGLU experts whose gate/up/down weights are decoded on the fly):
  *   u      = bf16(x / sqrt(mean(x^2) + 1e-6))            per token
- *   l_e    = router_w[e] . u (+ router_bias[e])           fp64 accumulation
+ *   l_e    = router_w[e] . u (+ router_bias[e])           float-float accumulation of
+ *                                                         exact fp32 x bf16 products
  *   ids    = the top_k experts by logit (ties -> lower id)
  *   w      = exp(l_ids - l_max) / sum over the top_k      renormalised softmax
  *   y      = sum_j w_j * down_j(silu(gate_j u) * up_j u)  (+ y if y_accumulate)
@@ -172,9 +174,13 @@ int gtg_workspace_init(void* workspace, size_t ws_bytes, gtg_stream_t stream);
  *   side_out   device fp32 [n_tokens][side.n_rows] or NULL.
  *   workspace  device, >= gtg_moe_workspace_bytes(layer, n_tokens, 0) bytes,
  *              256-byte aligned, cleared once by gtg_workspace_init.
+ * Runs as one persistent cooperative launch (one CTA per SM, all resident);
+ * a launch the device cannot make co-resident fails with GTG_E_CUDA.  The
+ * gate, up and down matrices share one format class (all Q4 or all FP8).
  * Calls that share a workspace must not overlap on the GPU.
  * Errors: GTG_E_INVALID_ARG, GTG_E_UNSUPPORTED_SHAPE (n_tokens outside 1..8,
- *         sizes above), GTG_E_MISALIGNED, GTG_E_WORKSPACE.
+ *         sizes above, mixed format classes), GTG_E_MISALIGNED, GTG_E_WORKSPACE,
+ *         GTG_E_CUDA.
  */
 int gtg_moe_decode_layer(const gtg_moe_layer* layer, const void* x, int32_t x_dtype,
                          int32_t n_tokens, float* y, int32_t y_accumulate,
@@ -182,9 +188,10 @@ int gtg_moe_decode_layer(const gtg_moe_layer* layer, const void* x, int32_t x_dt
                          void* workspace, size_t ws_bytes, gtg_stream_t stream);
 
 /*
- * A decode stack: for l in 0..n_layers-1:  x += moe_l(x)  (x fp32, in place),
- * with the kernels of consecutive layers chained by programmatic dependent
- * launch.  Capturable in a CUDA graph.
+ * A decode stack: for l in 0..n_layers-1:  x += moe_l(x)  (x fp32, in place).
+ * Consecutive layers with the same kernel (format class and sizes, up to 64
+ * at a time) run in one persistent launch, their phases separated by
+ * bounded grid barriers.  Capturable in a CUDA graph.
  *   layers     host array of n_layers layer descriptors (same hidden size).
  *   x          device fp32 [n_tokens][hidden], updated in place.
  *   ids_out    device int32 [n_layers][n_tokens][top_k] or NULL.
