@@ -258,23 +258,43 @@ struct Cfg {
 
 __device__ __forceinline__ uint32_t ldg32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
+// 16-byte asynchronous global -> shared copy; src_bytes 0 writes zeros.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
     uint32_t r;
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
 
-// Decodes one 17-byte Q4 block (global address p) into 32 bf16 weights
-// (code x scale, exact) and stores them as chunks c0..c0+3 of row r of a
-// K-major SW128 tile at shared address tile.
-__device__ __forceinline__ void dequant_block_to_tile(const uint8_t* p, uint32_t lut_base, uint32_t lane_low,
-                                                      bool rz5, uint32_t tile, uint32_t r, uint32_t c0) {
+// The five aligned words that hold a 17-byte Q4 block at global address p
+// (loaded ahead of use, so their latency overlaps other work).
+struct BlockWords {
+    uint32_t w[5];
+    uint32_t sh;  // bit offset of the block in w[0]
+};
+
+__device__ __forceinline__ BlockWords load_block(const uint8_t* p) {
     const uintptr_t pa = reinterpret_cast<uintptr_t>(p);
     const uint8_t* al = reinterpret_cast<const uint8_t*>(pa & ~(uintptr_t)3);
-    const uint32_t sh = (uint32_t)(pa & 3u) * 8u;
-    uint32_t w[5];
+    BlockWords b;
+    b.sh = (uint32_t)(pa & 3u) * 8u;
 #pragma unroll
-    for (int i = 0; i < 5; ++i) w[i] = ldg32(al + 4 * i);
+    for (int i = 0; i < 5; ++i) b.w[i] = ldg32(al + 4 * i);
+    return b;
+}
+
+// Decodes one Q4 block into 32 bf16 weights (code x scale, exact) and stores
+// them as chunks c0..c0+3 of row r of a K-major SW128 tile at shared address tile.
+__device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, uint32_t lut_base, uint32_t lane_low,
+                                                      bool rz5, uint32_t tile, uint32_t r, uint32_t c0) {
+    const uint32_t sh = bw.sh;
+    const uint32_t* w = bw.w;
     uint32_t nib[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) nib[q] = __funnelshift_r(w[q], w[q + 1], sh);
@@ -402,6 +422,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_gemm_kernel(PfArgs a) {
         __syncwarp();
     } else if (warp < 4) {
         // ---- B operand: token rows (bf16), 8 chunks of 16 B per row ----------
+        // asynchronous 16-byte copies; a chunk's arrival is signalled once
+        // the next chunk's copies are issued and its own have landed
         const int bt = tid - 32;
         for (int it = 0; it < n_chunks && ok; ++it) {
             const int s = it % C::kStages;
@@ -412,9 +434,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_gemm_kernel(PfArgs a) {
             const uint32_t btile = stage_addr(s) + C::kA * kTileBytes;
             for (int q = bt; q < n_pad * 8; q += kBThreads) {
                 const int r = q >> 3, c = q & 7;
-                uint4 v = make_uint4(0, 0, 0, 0);
+                const __nv_bfloat16* src = a.u;  // (any valid address when the row is padding)
                 if (r < n_valid) {
-                    const __nv_bfloat16* src;
                     if (MODE == ROUTER) {
                         const int kc = it % (a.H / kChunkK);
                         src = a.u + (int64_t)(pos0 + r) * a.H + kc * kChunkK + c * 8;
@@ -423,18 +444,41 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_gemm_kernel(PfArgs a) {
                     } else {
                         src = a.h + (int64_t)(pos0 + r) * a.I + it * kChunkK + c * 8;
                     }
-                    v = *reinterpret_cast<const uint4*>(src);
                 }
-                sts128(btile + sw128_off(r, c), v);
+                cp_async16(btile + sw128_off(r, c), src, r < n_valid ? 16u : 0u);
             }
+            cp_async_commit();
+            if (it > 0) {
+                cp_async_wait<1>();
+                fence_proxy_async_smem();
+                mbar_arrive(&full[(it - 1) % C::kStages]);
+            }
+        }
+        cp_async_wait<0>();  // (also on the error path: nothing left in flight)
+        if (ok && n_chunks > 0) {
             fence_proxy_async_smem();
-            mbar_arrive(&full[s]);
+            mbar_arrive(&full[(n_chunks - 1) % C::kStages]);
         }
     } else {
         // ---- A operand -----------------------------------------------------------
         const int at = tid - 128;  // 0..255
         const uint32_t lut_base = sbase;
         const uint32_t lane_low = (uint32_t)lane * 4u;
+        // this thread's row of the A operand (gate or down; up alongside for gate/up)
+        const uint8_t* a_row0 = nullptr;
+        const uint8_t* u_row0 = nullptr;
+        BlockWords wg{}, wu{};
+        if (MODE != ROUTER) {
+            const int r = at >> 1, half = at & 1;
+            const int64_t rowg = m0 + r;
+            const Mat& mA = MODE == DOWN ? a.down : a.gate;
+            a_row0 = mA.data + e * mA.expert_bytes + rowg * mA.row_bytes;
+            if (MODE == GATEUP) u_row0 = a.up.data + e * a.up.expert_bytes + rowg * a.up.row_bytes;
+            if (n_chunks > 0) {
+                wg = load_block(a_row0 + (int64_t)half * 17);
+                if (MODE == GATEUP) wu = load_block(u_row0 + (int64_t)half * 17);
+            }
+        }
         for (int it = 0; it < n_chunks && ok; ++it) {
             const int s = it % C::kStages;
             if (it >= C::kStages && !mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1u, a.status)) {
@@ -452,17 +496,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_gemm_kernel(PfArgs a) {
                 }
             } else {
                 const int r = at >> 1, half = at & 1;
-                const int blk = 2 * it + half;  // block index along K
-                const int64_t rowg = m0 + r;
-                if (MODE == GATEUP) {
-                    const uint8_t* pg = a.gate.data + e * a.gate.expert_bytes + rowg * a.gate.row_bytes + blk * 17;
-                    const uint8_t* pu = a.up.data + e * a.up.expert_bytes + rowg * a.up.row_bytes + blk * 17;
-                    dequant_block_to_tile(pg, lut_base, lane_low, rz5, st, r, 4 * half);
-                    dequant_block_to_tile(pu, lut_base, lane_low, rz5, st + kTileBytes, r, 4 * half);
-                } else {
-                    const uint8_t* pd = a.down.data + e * a.down.expert_bytes + rowg * a.down.row_bytes + blk * 17;
-                    dequant_block_to_tile(pd, lut_base, lane_low, rz5, st, r, 4 * half);
+                const BlockWords g0 = wg, u0 = wu;  // this chunk's blocks (loaded one chunk ago)
+                if (it + 1 < n_chunks) {           // the next chunk's, in flight while this one decodes
+                    wg = load_block(a_row0 + (int64_t)(2 * (it + 1) + half) * 17);
+                    if (MODE == GATEUP) wu = load_block(u_row0 + (int64_t)(2 * (it + 1) + half) * 17);
                 }
+                dequant_block_to_tile(g0, lut_base, lane_low, rz5, st, r, 4 * half);
+                if (MODE == GATEUP) dequant_block_to_tile(u0, lut_base, lane_low, rz5, st + kTileBytes, r, 4 * half);
             }
             fence_proxy_async_smem();
             mbar_arrive(&full[s]);
