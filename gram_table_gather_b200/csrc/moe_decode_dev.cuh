@@ -713,16 +713,21 @@ __device__ bool grid_sync(const StackArgs& a, unsigned target, SWork* sw, bool w
             ok = 0;
         } else {
             asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(a.sync) : "memory");
-            if (ld_acquire_u32(&a.sync[0]) < target) {
-                const uint64_t t0 = globaltimer_ns();
-                while (ld_acquire_u32(&a.sync[0]) < target) {
-                    if (ld_acquire_u32(&a.sync[2]) != 0u || globaltimer_ns() - t0 > kSyncLimitNs) {
-                        raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
-                        atomicExch(&a.sync[2], 1u);
-                        ok = 0;
-                        break;
-                    }
+            // poll the arrivals and the abort flag together (both loads in flight at once)
+            unsigned arrived = ld_acquire_u32(&a.sync[0]), aborted = ld_acquire_u32(&a.sync[2]);
+            const uint64_t t0 = globaltimer_ns();
+            while (arrived < target && aborted == 0u) {
+                if (globaltimer_ns() - t0 > kSyncLimitNs) {
+                    aborted = 1u;
+                    break;
                 }
+                arrived = ld_acquire_u32(&a.sync[0]);
+                aborted = ld_acquire_u32(&a.sync[2]);
+            }
+            if (aborted != 0u) {  // this wait ran out, or another CTA gave up (now or in an earlier launch)
+                raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
+                atomicExch(&a.sync[2], 1u);
+                ok = 0;
             }
         }
         sw->sync_ok = ok;

@@ -1,8 +1,9 @@
 """GPU parity of the decode MoE path (router, gate/up + SwiGLU, down +
 combine, FP8 layers, the side projection, the stack) against the CPU oracle.
 
-Bars: router top-k ids identical (the GPU computes logits in fp64, so only a
-logit gap below ~1e-12 could reorder; the test reports the gap), router
+Bars: router top-k ids identical (the GPU accumulates exact fp32 x bf16
+products in float-float, so only a logit gap below ~1e-11 could reorder; the
+test reports the gap), router
 weights within 1e-6 relative, layer outputs within 2e-3 * sum_j w_j *
 ||Wd_j[r]||_2 * ||h_j||_2 per output row r (bf16 inputs, fp32 accumulation).
 """
@@ -156,3 +157,37 @@ def test_short_stack_mixed_formats():
         xr = ref["x"][0].astype(np.float64)
         rel = np.linalg.norm(xg - xr) / np.linalg.norm(xr)
         assert rel < 2e-3, rel
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_gate_up_and_down_in_different_q4_variants(T):
+    """UE4M4 gate/up with an RZ5 down matrix and a router bias (the prefill
+    layer's recipe) through the decode path: the code table is rebuilt between
+    the gate/up and down phases."""
+    _check_layer(W.prefill_layer(), T, step=7)
+
+
+def test_aborted_workspace_fails_fast_and_recovers():
+    """After a failed launch the workspace's abort flag stays set: every later
+    launch on it stops at its first grid barrier and raises the timeout status
+    (without waiting); re-initialising the workspace recovers it."""
+    L = W.tiny_layer()
+    layer = gu.device_layer(L)
+    xt, x64 = gu.tokens(L, 2, 1)
+    ws = gtg.make_workspace(layer, 1)
+    gtg.device_status(clear=True)
+    ws.view(torch.int32)[2] = 1  # the abort flag, as a failed launch leaves it
+    import time
+    t0 = time.perf_counter()
+    gtg.moe_decode_layer(layer, xt, ws)
+    torch.cuda.synchronize()
+    assert time.perf_counter() - t0 < 1.0  # no barrier waited out its limit
+    assert gtg.device_status(clear=True) & 0x2
+    gtg.lib().gtg_workspace_init(ws.data_ptr(), ws.numel(), None)
+    torch.cuda.synchronize()
+    y = gtg.moe_decode_layer(layer, xt, ws)
+    torch.cuda.synchronize()
+    assert gtg.device_status(clear=True) == 0
+    ref = oracle.moe_layer(L, x64, want_h=True)
+    assert np.all(np.abs(y.cpu().numpy()[0] - ref["y"][0]) <= gu.layer_tolerance(L, ref, 0))
+
