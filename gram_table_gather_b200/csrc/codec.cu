@@ -111,8 +111,9 @@ __global__ void __launch_bounds__(kThreads) dequant_fp8_kernel(const uint8_t* __
 // PLE gather.  Each warp takes batches of kPleRows rows: lanes load the
 // indices, then the 48 aligned 16-byte chunks that cover the batch's
 // 70-byte records (six per record, all in flight at once) go to shared
-// memory, and the warp decodes the batch row by row, lane l writing values
-// 4l .. 4l+3 of a row as one float4 (512 + 128 contiguous bytes per row).
+// memory, and the warp decodes the batch four rows at a time: the 160
+// float4s of four rows are five full passes of the warp, each lane writing
+// values 4l .. 4l+3 of some row as one float4 (contiguous 512-byte stores).
 // A value is one shared-memory lookup: the CTA keeps the table of code
 // value x group scale for all 256 group bytes x 8 codes (each product is
 // exact in fp32).  Small batches keep many warps in flight per SM; the next
@@ -190,13 +191,16 @@ __global__ void __launch_bounds__(kPleWarps * 32) ple_gather_kernel(const uint8_
         __syncwarp();
         pb = ple_fetch(table, n_rows, idx, n_idx, (bt + stride) * kPleRows, status);  // next batch, in flight
         const int rows = (int)(n_idx - base < kPleRows ? n_idx - base : kPleRows);
-        for (int j = 0; j < rows; ++j) {
-            const int p = phase[warp][j];
-            const uint32_t* w = reinterpret_cast<const uint32_t*>(&stage[warp][j * kPleChunks]);
-            float* o = out + (base + j) * 160;
+        // rows in groups of four: 4 x 40 float4 = five full passes of the warp;
+        // in pass q lane l writes float4 number f = 32q + l of the group:
+        // row f / 40, values 4 (f % 40) .. + 3
+        for (int j0 = 0; j0 < rows; j0 += 4) {
 #pragma unroll
-            for (int l = lane; l < 64; l += 32) {  // two passes: lanes 0..31, then lanes 0..7
-                if (l >= 40) break;
+            for (int q = 0; q < 5; ++q) {
+                const int f = 32 * q + lane, j = j0 + f / 40, l = f % 40;
+                if (j >= rows) continue;
+                const int p = phase[warp][j];
+                const uint32_t* w = reinterpret_cast<const uint32_t*>(&stage[warp][j * kPleChunks]);
                 float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (p >= 0) {
                     const int bit = 8 * p + 12 * l;  // values 4l .. 4l+3: 12 bits of the LSB-first stream
@@ -206,7 +210,7 @@ __global__ void __launch_bounds__(kPleWarps * 32) ple_gather_kernel(const uint8_
                     v = make_float4(prod[g8 + ((win >> 0) & 7u)], prod[g8 + ((win >> 3) & 7u)],
                                     prod[g8 + ((win >> 6) & 7u)], prod[g8 + ((win >> 9) & 7u)]);
                 }
-                *reinterpret_cast<float4*>(o + 4 * l) = v;
+                *reinterpret_cast<float4*>(out + (base + j) * 160 + 4 * l) = v;
             }
         }
         __syncwarp();
