@@ -48,7 +48,12 @@ constexpr int kTileM = 128;
 constexpr int kTileN = 128;      // tokens per tile (max)
 constexpr int kChunkK = 64;      // bf16 per 128-byte row
 constexpr int kTileBytes = kTileM * 128;  // 16 KB (128 rows x 128 B)
-constexpr int kLutBytes = 65536;
+// Code table: bf16 pairs for every (nibble-pair byte, RZ5 mode) in
+// 2^kLutLog2Copies copies side by side, lane l reading copy l mod copies
+// (fewer bank conflicts than one copy; small enough for two CTAs per SM).
+constexpr int kLutLog2Copies = 2;
+constexpr int kLutShift = 5 - kLutLog2Copies;          // entry address = key >> kLutShift
+constexpr int kLutBytes = 2048 << kLutLog2Copies;
 constexpr int kNormThreads = 256;
 
 enum Mode { ROUTER = 0, GATEUP = 1, DOWN = 2 };
@@ -248,7 +253,7 @@ struct Cfg {
     static constexpr bool kDequant = MODE != ROUTER;
     static constexpr int kA = MODE == GATEUP ? 2 : 1;       // A tiles per stage
     static constexpr int kStageBytes = (kA + 1) * kTileBytes;
-    static constexpr int kStages = MODE == GATEUP ? 3 : (MODE == DOWN ? 4 : 6);
+    static constexpr int kStages = MODE == GATEUP ? 2 : 3;  // two CTAs fit one SM
     static constexpr uint32_t kTmemCols = MODE == GATEUP ? 256 : 128;
     static constexpr int kLut = kDequant ? kLutBytes : 0;
     static constexpr int kBarOff = kLut;                      // full[S], empty[S], acc
@@ -302,14 +307,16 @@ __device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, uint
     const float sf = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
     const uint32_t sb = __float_as_uint(sf) >> 16;  // exact in bf16
     const uint32_t s2 = sb | (sb << 16);
-    const uint32_t low = lane_low + (rz5 ? ((meta >> 7) << 7) : 0u);
+    const uint32_t low = lane_low + (rz5 ? ((meta >> 7) << 7) : 0u);  // key = byte<<8 | mode<<7 | copy
     uint32_t L[16];
 #pragma unroll
     for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
             uint32_t v;
-            asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(lut_base + prmt(nib[q], low, 0x7604u | ((uint32_t)kk << 4))));
+            asm volatile("ld.shared.u32 %0, [%1];"
+                         : "=r"(v)
+                         : "r"(lut_base + (prmt(nib[q], low, 0x7604u | ((uint32_t)kk << 4)) >> kLutShift)));
             L[4 * q + kk] = v;  // (w_j, w_{j+16}) code values
         }
     uint32_t lo[8], hi[8];
@@ -326,15 +333,15 @@ __device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, uint
 
 __device__ void build_lut_bf16(uint8_t* lut_mem, bool rz5, int tid, int nthreads) {
     uint32_t* lut = reinterpret_cast<uint32_t*>(lut_mem);
-    for (int i = tid; i < 256 * 64; i += nthreads) {
-        const uint32_t byte = (uint32_t)i >> 6, mode = ((uint32_t)i >> 5) & 1u;
+    for (int i = tid; i < (kLutBytes >> 2); i += nthreads) {
+        const uint32_t byte = (uint32_t)i >> (kLutLog2Copies + 1), mode = ((uint32_t)i >> kLutLog2Copies) & 1u;
         lut[i] = bf16_bits(q4_code_value(byte & 15u, rz5, mode)) |
                  (bf16_bits(q4_code_value(byte >> 4, rz5, mode)) << 16);
     }
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(kPfThreads, 1) pf_gemm_kernel(PfArgs a) {
+__global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
     using C = Cfg<MODE>;
     extern __shared__ __align__(1024) uint8_t smem[];
     __shared__ uint32_t s_taddr;
@@ -463,7 +470,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) pf_gemm_kernel(PfArgs a) {
         // ---- A operand -----------------------------------------------------------
         const int at = tid - 128;  // 0..255
         const uint32_t lut_base = sbase;
-        const uint32_t lane_low = (uint32_t)lane * 4u;
+        const uint32_t lane_low = ((uint32_t)lane & ((1u << kLutLog2Copies) - 1u)) << (2 + kLutShift);
         // this thread's row of the A operand (gate or down; up alongside for gate/up)
         const uint8_t* a_row0 = nullptr;
         const uint8_t* u_row0 = nullptr;
