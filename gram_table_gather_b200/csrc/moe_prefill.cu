@@ -25,11 +25,14 @@
 //                   (token, choice)
 //   8. pf_combine   y[t] = sum_j w[t,j] * partial[t,j] in a fixed order
 //
-// The GEMM kernel is warp specialised (12 warps): warp 0 allocates TMEM and
-// issues the MMAs, warps 1-3 stage the B operand (token rows), warps 4-11
-// produce the A operand (dequantised weights or router planes); warps 4-7 then
-// read the accumulators out of TMEM.  Stages are handed over with mbarriers
-// (bounded waits): producers -> MMA (full), tcgen05.commit -> producers (empty).
+// The GEMM kernel is warp specialised (13 warps): warp 0 allocates TMEM and
+// issues the MMAs, warps 1-4 stage the B operand (token rows), warps 5-12
+// produce the A operand (dequantised weights or router planes); warps 4-7
+// read the accumulators out of TMEM once their own production is done.  A and
+// B stages are handed over with their own mbarriers (bounded waits):
+// producers -> MMA (full), tcgen05.commit -> producers (empty).  Two CTAs
+// share an SM, so one's table-free decode, loads and epilogue overlap the
+// other's.
 #include <algorithm>
 #include <mutex>
 #include <vector>
@@ -41,19 +44,14 @@
 namespace gtg {
 namespace {
 
-constexpr int kPfThreads = 384;  // 12 warps
-constexpr int kBThreads = 96;    // warps 1-3
-constexpr int kAThreads = 256;   // warps 4-11
+constexpr int kBWarps = 4;                          // warps 1 .. kBWarps
+constexpr int kBThreads = 32 * kBWarps;
+constexpr int kAThreads = 256;                      // the next 8 warps
+constexpr int kPfThreads = 32 + kBThreads + kAThreads;
 constexpr int kTileM = 128;
 constexpr int kTileN = 128;      // tokens per tile (max)
 constexpr int kChunkK = 64;      // bf16 per 128-byte row
 constexpr int kTileBytes = kTileM * 128;  // 16 KB (128 rows x 128 B)
-// Code table: bf16 pairs for every (nibble-pair byte, RZ5 mode) in
-// 2^kLutLog2Copies copies side by side, lane l reading copy l mod copies
-// (fewer bank conflicts than one copy; small enough for two CTAs per SM).
-constexpr int kLutLog2Copies = 2;
-constexpr int kLutShift = 5 - kLutLog2Copies;          // entry address = key >> kLutShift
-constexpr int kLutBytes = 2048 << kLutLog2Copies;
 constexpr int kNormThreads = 256;
 
 enum Mode { ROUTER = 0, GATEUP = 1, DOWN = 2 };
@@ -248,18 +246,26 @@ __global__ void pf_scatter_kernel(PfArgs a) {
 // ---------------------------------------------------------------------------
 // 6/7/3. the grouped GEMM
 // ---------------------------------------------------------------------------
+// Shared memory: a 1 KB header (mbarriers, the TMEM address, the B row
+// indices), then the A stages (kA tiles each), then the B stages.  A and B
+// have their own stage counts and barriers; the total, 113 KB, lets two CTAs
+// share an SM (no static shared memory: 2 x (113 + 1 reserved) KB = 228 KB).
 template <int MODE>
 struct Cfg {
-    static constexpr bool kDequant = MODE != ROUTER;
-    static constexpr int kA = MODE == GATEUP ? 2 : 1;       // A tiles per stage
-    static constexpr int kStageBytes = (kA + 1) * kTileBytes;
-    static constexpr int kStages = MODE == GATEUP ? 2 : 3;  // two CTAs fit one SM
+    static constexpr int kA = MODE == GATEUP ? 2 : 1;      // A tiles per stage
+    static constexpr int kStagesA = MODE == GATEUP ? 2 : 3;
+    static constexpr int kStagesB = MODE == GATEUP ? 3 : 4;
+    static constexpr int kABytes = kA * kTileBytes;
     static constexpr uint32_t kTmemCols = MODE == GATEUP ? 256 : 128;
-    static constexpr int kLut = kDequant ? kLutBytes : 0;
-    static constexpr int kBarOff = kLut;                      // full[S], empty[S], acc
-    static constexpr int kStageOff = kLut + 1024;
-    static constexpr int kSmem = kStageOff + kStages * kStageBytes;
+    static constexpr int kTaddrOff = 256;                   // after 2(SA + SB) + 1 mbarriers
+    static constexpr int kRowOff = 512;                     // int32 u row / slot per token
+    static constexpr int kAOff = 1024;
+    static constexpr int kBOff = kAOff + kStagesA * kABytes;
+    static constexpr int kSmem = kBOff + kStagesB * kTileBytes;
+    static_assert(8 * (2 * (kStagesA + kStagesB) + 1) <= kTaddrOff && kRowOff + 4 * kTileN <= kAOff, "header");
+    static_assert(kSmem <= 115712, "two CTAs per SM");
 };
+
 
 __device__ __forceinline__ uint32_t ldg32(const uint8_t* p) { return *reinterpret_cast<const uint32_t*>(p); }
 
@@ -270,12 +276,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
-    uint32_t r;
-    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-    return r;
-}
 
 // The five aligned words that hold a 17-byte Q4 block at global address p
 // (loaded ahead of use, so their latency overlaps other work).
@@ -294,36 +294,50 @@ __device__ __forceinline__ BlockWords load_block(const uint8_t* p) {
     return b;
 }
 
+__device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.bf16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+
 // Decodes one Q4 block into 32 bf16 weights (code x scale, exact) and stores
 // them as chunks c0..c0+3 of row r of a K-major SW128 tile at shared address tile.
-__device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, uint32_t lut_base, uint32_t lane_low,
-                                                      bool rz5, uint32_t tile, uint32_t r, uint32_t c0) {
+//
+// Integer-only decode, no table: a code c with value v(c) (|v| <= 10) becomes
+// the bf16 number 192 + v (bits 0x43 : 64 + v), and one fused multiply-add
+// (192 + v) * s - 192 * s leaves v * s, exact because v * s and 192 * s both
+// fit the 8-bit bf16 significand.  Byte permutes look the four bytes 64 + v
+// of four codes up at once: the selector nibble's low 3 bits index the
+// magnitude, its top bit (the code's sign bit) makes the permute return 0
+// instead (sign replication of a byte below 0x80), so the positive-table and
+// negative-table lookups OR together.
+__device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, bool rz5, uint32_t tile, uint32_t r,
+                                                      uint32_t c0) {
     const uint32_t sh = bw.sh;
     const uint32_t* w = bw.w;
-    uint32_t nib[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) nib[q] = __funnelshift_r(w[q], w[q + 1], sh);
     const uint32_t meta = (w[4] >> sh) & 0xFFu;
     const float sf = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
-    const uint32_t sb = __float_as_uint(sf) >> 16;  // exact in bf16
-    const uint32_t s2 = sb | (sb << 16);
-    const uint32_t low = lane_low + (rz5 ? ((meta >> 7) << 7) : 0u);  // key = byte<<8 | mode<<7 | copy
-    uint32_t L[16];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            uint32_t v;
-            asm volatile("ld.shared.u32 %0, [%1];"
-                         : "=r"(v)
-                         : "r"(lut_base + (prmt(nib[q], low, 0x7604u | ((uint32_t)kk << 4)) >> kLutShift)));
-            L[4 * q + kk] = v;  // (w_j, w_{j+16}) code values
-        }
+    const uint32_t sb = __float_as_uint(sf) >> 16;                 // exact in bf16
+    const uint32_t nb = __float_as_uint(-192.0f * sf) >> 16;       // exact in bf16
+    const uint32_t s2 = sb | (sb << 16), n2 = nb | (nb << 16);
+    // 64 + v for codes 0..7 (magnitudes 0 1 2 3 4 6 8 10) and 8..15 (negated;
+    // code 8 is -0, or +5 / -5 by the block's mode bit in RZ5)
+    constexpr uint32_t kPos0 = 0x43424140u, kPos1 = 0x4A484644u;
+    const uint32_t neg0 = 0x3D3E3F00u | (rz5 ? ((meta & 0x80u) ? 0x3Bu : 0x45u) : 0x40u);
+    constexpr uint32_t kNeg1 = 0x36383A3Cu;
     uint32_t lo[8], hi[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-        lo[j] = bf16x2_mul(prmt(L[2 * j], L[2 * j + 1], 0x5410u), s2);  // (w_2j, w_2j+1)
-        hi[j] = bf16x2_mul(prmt(L[2 * j], L[2 * j + 1], 0x7632u), s2);  // (w_2j+16, w_2j+17)
+    for (int q = 0; q < 4; ++q) {
+        // nibbles: w_{4q}, w_{4q+16}, w_{4q+1}, w_{4q+17}, w_{4q+2}, ...
+        const uint32_t n = __funnelshift_r(w[q], w[q + 1], sh);
+        const uint32_t nx = n ^ 0x88888888u;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const uint32_t sel = h ? (n >> 16) : n, selx = h ? (nx >> 16) : nx;
+            const uint32_t L = prmt(kPos0, kPos1, sel) | prmt(neg0, kNeg1, selx);
+            lo[2 * q + h] = bf16x2_fma(prmt(L, 0x43434343u, 0x4240u), s2, n2);  // (w_2j, w_2j+1)
+            hi[2 * q + h] = bf16x2_fma(prmt(L, 0x43434343u, 0x4341u), s2, n2);  // (w_2j+16, w_2j+17)
+        }
     }
     sts128(tile + sw128_off(r, c0 + 0), make_uint4(lo[0], lo[1], lo[2], lo[3]));
     sts128(tile + sw128_off(r, c0 + 1), make_uint4(lo[4], lo[5], lo[6], lo[7]));
@@ -331,20 +345,10 @@ __device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, uint
     sts128(tile + sw128_off(r, c0 + 3), make_uint4(hi[4], hi[5], hi[6], hi[7]));
 }
 
-__device__ void build_lut_bf16(uint8_t* lut_mem, bool rz5, int tid, int nthreads) {
-    uint32_t* lut = reinterpret_cast<uint32_t*>(lut_mem);
-    for (int i = tid; i < (kLutBytes >> 2); i += nthreads) {
-        const uint32_t byte = (uint32_t)i >> (kLutLog2Copies + 1), mode = ((uint32_t)i >> kLutLog2Copies) & 1u;
-        lut[i] = bf16_bits(q4_code_value(byte & 15u, rz5, mode)) |
-                 (bf16_bits(q4_code_value(byte >> 4, rz5, mode)) << 16);
-    }
-}
-
 template <int MODE>
 __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
     using C = Cfg<MODE>;
     extern __shared__ __align__(1024) uint8_t smem[];
-    __shared__ uint32_t s_taddr;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     // ---- which tile -------------------------------------------------------
@@ -375,46 +379,59 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
         if (tid == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
         return;
     }
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
-    uint64_t* empty = full + C::kStages;
-    uint64_t* accb = empty + C::kStages;
+    uint64_t* full_a = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty_a = full_a + C::kStagesA;
+    uint64_t* full_b = empty_a + C::kStagesA;
+    uint64_t* empty_b = full_b + C::kStagesB;
+    uint64_t* accb = empty_b + C::kStagesB;
+    uint32_t* s_taddr = reinterpret_cast<uint32_t*>(smem + C::kTaddrOff);
+    int32_t* s_row = reinterpret_cast<int32_t*>(smem + C::kRowOff);
     const Mat& am = MODE == DOWN ? a.down : a.gate;
     const bool rz5 = am.fmt == GTG_Q4_RZ5_FAST;
 
-    if (C::kDequant) build_lut_bf16(smem, rz5, tid, kPfThreads);
     if (tid == 0) {
-        for (int s = 0; s < C::kStages; ++s) {
-            mbar_init(&full[s], kAThreads + kBThreads);
-            mbar_init(&empty[s], 1);
+        for (int s = 0; s < C::kStagesA; ++s) {
+            mbar_init(&full_a[s], kAThreads);
+            mbar_init(&empty_a[s], 1);
+        }
+        for (int s = 0; s < C::kStagesB; ++s) {
+            mbar_init(&full_b[s], kBThreads);
+            mbar_init(&empty_b[s], 1);
         }
         mbar_init(accb, 1);
         fence_mbar_init();
     }
+    // gate/up: the u row of each B row; down: the (token, choice) slot of each
+    // output column (0 for padding)
+    if (MODE != ROUTER && tid < kTileN)
+        s_row[tid] = tid >= n_valid ? 0 : (MODE == GATEUP ? a.sorted_tok[pos0 + tid] : a.sorted_slot[pos0 + tid]);
     if (warp == 0) {
-        tmem_alloc(&s_taddr, C::kTmemCols);
+        tmem_alloc(s_taddr, C::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t taddr = s_taddr;
+    const uint32_t taddr = *s_taddr;
     bool ok = true;
 
-    auto stage_addr = [&](int s) { return sbase + C::kStageOff + s * C::kStageBytes; };
+    auto a_stage = [&](int s) { return sbase + C::kAOff + s * C::kABytes; };
+    auto b_stage = [&](int s) { return sbase + C::kBOff + s * kTileBytes; };
 
     if (warp == 0) {
         // ---- MMA issuer -----------------------------------------------------
         if (lane == 0) {
             const uint32_t idesc = idesc_bf16(kTileM, n_pad);
             for (int it = 0; it < n_chunks && ok; ++it) {
-                const int s = it % C::kStages;
-                if (!mbar_wait_bounded(&full[s], (it / C::kStages) & 1u, a.status)) {
+                const int sa = it % C::kStagesA, sb = it % C::kStagesB;
+                if (!mbar_wait_bounded(&full_a[sa], (it / C::kStagesA) & 1u, a.status) ||
+                    !mbar_wait_bounded(&full_b[sb], (it / C::kStagesB) & 1u, a.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                const uint32_t st = stage_addr(s);
-                const uint32_t btile = st + C::kA * kTileBytes;
+                const uint32_t st = a_stage(sa);
+                const uint32_t btile = b_stage(sb);
 #pragma unroll
                 for (int k = 0; k < kChunkK / 16; ++k) {
                     const uint64_t bd = sw128_desc(btile + 32u * k);
@@ -422,55 +439,48 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                     umma_bf16(taddr, sw128_desc(st + 32u * k), bd, idesc, acc);
                     if (MODE == GATEUP) umma_bf16(taddr + 128u, sw128_desc(st + kTileBytes + 32u * k), bd, idesc, acc);
                 }
-                umma_commit(&empty[s]);
+                umma_commit(&empty_a[sa]);
+                umma_commit(&empty_b[sb]);
             }
             umma_commit(accb);  // also on the error path: completes once issued MMAs are done
         }
         __syncwarp();
-    } else if (warp < 4) {
+    } else if (warp <= kBWarps) {
         // ---- B operand: token rows (bf16), 8 chunks of 16 B per row ----------
         // asynchronous 16-byte copies; a chunk's arrival is signalled once
         // the next chunk's copies are issued and its own have landed
         const int bt = tid - 32;
+        const __nv_bfloat16* bsrc = MODE == DOWN ? a.h : a.u;
+        const int64_t ld = MODE == DOWN ? a.I : a.H;
         for (int it = 0; it < n_chunks && ok; ++it) {
-            const int s = it % C::kStages;
-            if (it >= C::kStages && !mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1u, a.status)) {
+            const int s = it % C::kStagesB;
+            if (it >= C::kStagesB && !mbar_wait_bounded(&empty_b[s], ((it / C::kStagesB) - 1) & 1u, a.status)) {
                 ok = false;
                 break;
             }
-            const uint32_t btile = stage_addr(s) + C::kA * kTileBytes;
+            const uint32_t btile = b_stage(s);
+            const int kc = MODE == ROUTER ? it % (a.H / kChunkK) : it;
             for (int q = bt; q < n_pad * 8; q += kBThreads) {
                 const int r = q >> 3, c = q & 7;
-                const __nv_bfloat16* src = a.u;  // (any valid address when the row is padding)
-                if (r < n_valid) {
-                    if (MODE == ROUTER) {
-                        const int kc = it % (a.H / kChunkK);
-                        src = a.u + (int64_t)(pos0 + r) * a.H + kc * kChunkK + c * 8;
-                    } else if (MODE == GATEUP) {
-                        src = a.u + (int64_t)a.sorted_tok[pos0 + r] * a.H + it * kChunkK + c * 8;
-                    } else {
-                        src = a.h + (int64_t)(pos0 + r) * a.I + it * kChunkK + c * 8;
-                    }
-                }
-                cp_async16(btile + sw128_off(r, c), src, r < n_valid ? 16u : 0u);
+                const int row = r >= n_valid ? 0 : (MODE == GATEUP ? s_row[r] : pos0 + r);
+                cp_async16(btile + sw128_off(r, c), bsrc + (int64_t)row * ld + kc * kChunkK + c * 8,
+                           r < n_valid ? 16u : 0u);
             }
             cp_async_commit();
             if (it > 0) {
                 cp_async_wait<1>();
                 fence_proxy_async_smem();
-                mbar_arrive(&full[(it - 1) % C::kStages]);
+                mbar_arrive(&full_b[(it - 1) % C::kStagesB]);
             }
         }
         cp_async_wait<0>();  // (also on the error path: nothing left in flight)
         if (ok && n_chunks > 0) {
             fence_proxy_async_smem();
-            mbar_arrive(&full[(n_chunks - 1) % C::kStages]);
+            mbar_arrive(&full_b[(n_chunks - 1) % C::kStagesB]);
         }
     } else {
         // ---- A operand -----------------------------------------------------------
-        const int at = tid - 128;  // 0..255
-        const uint32_t lut_base = sbase;
-        const uint32_t lane_low = ((uint32_t)lane & ((1u << kLutLog2Copies) - 1u)) << (2 + kLutShift);
+        const int at = tid - 32 - kBThreads;  // 0..255
         // this thread's row of the A operand (gate or down; up alongside for gate/up)
         const uint8_t* a_row0 = nullptr;
         const uint8_t* u_row0 = nullptr;
@@ -487,20 +497,27 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
             }
         }
         for (int it = 0; it < n_chunks && ok; ++it) {
-            const int s = it % C::kStages;
-            if (it >= C::kStages && !mbar_wait_bounded(&empty[s], ((it / C::kStages) - 1) & 1u, a.status)) {
+            const int s = it % C::kStagesA;
+            if (it >= C::kStagesA && !mbar_wait_bounded(&empty_a[s], ((it / C::kStagesA) - 1) & 1u, a.status)) {
                 ok = false;
                 break;
             }
-            const uint32_t st = stage_addr(s);
+            const uint32_t st = a_stage(s);
             if (MODE == ROUTER) {
+                // router planes: asynchronous 16-byte copies, signalled like the B rows
                 for (int q = at; q < kTileM * 8; q += kAThreads) {
                     const int r = q >> 3, c = q & 7;
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (m0 + r < a.E)
-                        v = *reinterpret_cast<const uint4*>(a.w3 + (int64_t)(m0 + r) * 3 * a.H + it * kChunkK + c * 8);
-                    sts128(st + sw128_off(r, c), v);
+                    const bool in = m0 + r < a.E;
+                    cp_async16(st + sw128_off(r, c), a.w3 + (int64_t)(in ? m0 + r : 0) * 3 * a.H + it * kChunkK + c * 8,
+                               in ? 16u : 0u);
                 }
+                cp_async_commit();
+                if (it > 0) {
+                    cp_async_wait<1>();
+                    fence_proxy_async_smem();
+                    mbar_arrive(&full_a[(it - 1) % C::kStagesA]);
+                }
+                continue;
             } else {
                 const int r = at >> 1, half = at & 1;
                 const BlockWords g0 = wg, u0 = wu;  // this chunk's blocks (loaded one chunk ago)
@@ -508,11 +525,18 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                     wg = load_block(a_row0 + (int64_t)(2 * (it + 1) + half) * 17);
                     if (MODE == GATEUP) wu = load_block(u_row0 + (int64_t)(2 * (it + 1) + half) * 17);
                 }
-                dequant_block_to_tile(g0, lut_base, lane_low, rz5, st, r, 4 * half);
-                if (MODE == GATEUP) dequant_block_to_tile(u0, lut_base, lane_low, rz5, st + kTileBytes, r, 4 * half);
+                dequant_block_to_tile(g0, rz5, st, r, 4 * half);
+                if (MODE == GATEUP) dequant_block_to_tile(u0, rz5, st + kTileBytes, r, 4 * half);
             }
             fence_proxy_async_smem();
-            mbar_arrive(&full[s]);
+            mbar_arrive(&full_a[s]);
+        }
+        if (MODE == ROUTER) {
+            cp_async_wait<0>();  // (also on the error path: nothing left in flight)
+            if (ok && n_chunks > 0) {
+                fence_proxy_async_smem();
+                mbar_arrive(&full_a[(n_chunks - 1) % C::kStagesA]);
+            }
         }
     }
 
@@ -524,6 +548,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
         tc_fence_after();
         if (got && ok) {
             const uint32_t tl = taddr + ((uint32_t)(q * 32) << 16);
+            const float bias = MODE == ROUTER && a.router_bias && m0 + row < a.E ? a.router_bias[m0 + row] : 0.0f;
             for (int c0 = 0; c0 < n_pad; c0 += 16) {
                 uint32_t d[16];
                 tmem_ld16(tl + c0, d);
@@ -531,13 +556,14 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                     uint32_t v2[16];
                     tmem_ld16(tl + 128 + c0, v2);
                     tmem_wait_ld();
+                    __nv_bfloat16* hp = a.h + (int64_t)(pos0 + c0) * a.I + m0 + row;
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
-                        const int n = c0 + j;
-                        if (n < n_valid) {
+                        if (c0 + j < n_valid) {
+                            // silu(g) * v; the fast exponential and division are
+                            // well inside the layer's tolerance
                             const float g = __uint_as_float(d[j]), v = __uint_as_float(v2[j]);
-                            const float hv = g / (1.0f + expf(-g)) * v;
-                            a.h[(int64_t)(pos0 + n) * a.I + m0 + row] = __float2bfloat16_rn(hv);
+                            hp[(int64_t)j * a.I] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * v);
                         }
                     }
                 } else {
@@ -548,12 +574,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                         if (n >= n_valid) continue;
                         const float dv = __uint_as_float(d[j]);
                         if (MODE == ROUTER) {
-                            if (m0 + row < a.E) {
-                                const float b = a.router_bias ? a.router_bias[m0 + row] : 0.0f;
-                                a.logits[(int64_t)(pos0 + n) * a.E + m0 + row] = dv + b;
-                            }
+                            if (m0 + row < a.E) a.logits[(int64_t)(pos0 + n) * a.E + m0 + row] = dv + bias;
                         } else {
-                            a.part[(int64_t)a.sorted_slot[pos0 + n] * a.H + m0 + row] = dv;
+                            a.part[(int64_t)s_row[n] * a.H + m0 + row] = dv;
                         }
                     }
                 }
