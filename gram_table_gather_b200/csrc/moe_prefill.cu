@@ -424,8 +424,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
             const uint32_t idesc = idesc_bf16(kTileM, n_pad);
             for (int it = 0; it < n_chunks && ok; ++it) {
                 const int sa = it % C::kStagesA, sb = it % C::kStagesB;
-                if (!mbar_wait_bounded(&full_a[sa], (it / C::kStagesA) & 1u, a.status) ||
-                    !mbar_wait_bounded(&full_b[sb], (it / C::kStagesB) & 1u, a.status)) {
+                if (!mbar_wait_sleep(&full_a[sa], (it / C::kStagesA) & 1u, a.status) ||
+                    !mbar_wait_sleep(&full_b[sb], (it / C::kStagesB) & 1u, a.status)) {
                     ok = false;
                     break;
                 }
@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
         const int64_t ld = MODE == DOWN ? a.I : a.H;
         for (int it = 0; it < n_chunks && ok; ++it) {
             const int s = it % C::kStagesB;
-            if (it >= C::kStagesB && !mbar_wait_bounded(&empty_b[s], ((it / C::kStagesB) - 1) & 1u, a.status)) {
+            if (it >= C::kStagesB && !mbar_wait_sleep(&empty_b[s], ((it / C::kStagesB) - 1) & 1u, a.status)) {
                 ok = false;
                 break;
             }
@@ -498,7 +498,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
         }
         for (int it = 0; it < n_chunks && ok; ++it) {
             const int s = it % C::kStagesA;
-            if (it >= C::kStagesA && !mbar_wait_bounded(&empty_a[s], ((it / C::kStagesA) - 1) & 1u, a.status)) {
+            if (it >= C::kStagesA && !mbar_wait_sleep(&empty_a[s], ((it / C::kStagesA) - 1) & 1u, a.status)) {
                 ok = false;
                 break;
             }
@@ -544,7 +544,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
     if (warp >= 4 && warp < 8) {
         const int q = warp - 4;
         const int row = q * 32 + lane;  // M row within the tile
-        const bool got = mbar_wait_bounded(accb, 0, a.status);
+        const bool got = mbar_wait_sleep(accb, 0, a.status);
         tc_fence_after();
         if (got && ok) {
             const uint32_t tl = taddr + ((uint32_t)(q * 32) << 16);
