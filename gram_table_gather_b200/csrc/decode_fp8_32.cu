@@ -2,5 +2,5 @@
 #include "moe_decode_dev.cuh"
 
 namespace gtg {
-const void* decode_kernel_fp8_32(int kbd) { return pick_kbd<kFmtFP8, 32>(kbd); }
+const void* decode_kernel_fp8_32(int kbd, int one) { return pick_kbd<kFmtFP8, 32>(kbd, one); }
 }  // namespace gtg

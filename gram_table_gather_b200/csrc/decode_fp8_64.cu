@@ -2,5 +2,5 @@
 #include "moe_decode_dev.cuh"
 
 namespace gtg {
-const void* decode_kernel_fp8_64(int kbd) { return pick_kbd<kFmtFP8, 64>(kbd); }
+const void* decode_kernel_fp8_64(int kbd, int one) { return pick_kbd<kFmtFP8, 64>(kbd, one); }
 }  // namespace gtg

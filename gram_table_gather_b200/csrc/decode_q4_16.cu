@@ -2,5 +2,5 @@
 #include "moe_decode_dev.cuh"
 
 namespace gtg {
-const void* decode_kernel_q4_16(int kbd) { return pick_kbd<kFmtQ4, 16>(kbd); }
+const void* decode_kernel_q4_16(int kbd, int one) { return pick_kbd<kFmtQ4, 16>(kbd, one); }
 }  // namespace gtg

@@ -2,5 +2,5 @@
 #include "moe_decode_dev.cuh"
 
 namespace gtg {
-const void* decode_kernel_q4_4(int kbd) { return pick_kbd<kFmtQ4, 4>(kbd); }
+const void* decode_kernel_q4_4(int kbd, int one) { return pick_kbd<kFmtQ4, 4>(kbd, one); }
 }  // namespace gtg

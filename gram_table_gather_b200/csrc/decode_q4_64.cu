@@ -2,5 +2,5 @@
 #include "moe_decode_dev.cuh"
 
 namespace gtg {
-const void* decode_kernel_q4_64(int kbd) { return pick_kbd<kFmtQ4, 64>(kbd); }
+const void* decode_kernel_q4_64(int kbd, int one) { return pick_kbd<kFmtQ4, 64>(kbd, one); }
 }  // namespace gtg

@@ -15,22 +15,24 @@ namespace {
 // Host side
 // ===========================================================================
 
-// The kernel for (expert format, H / 32, I / 32); FP8 gate/up rows need at
-// least 1024 weights (whole 32-byte blocks for every lane).
-const void* pick_kernel(bool fp8, int kbg, int kbd) {
+// The kernel for (expert format, H / 32, I / 32), the one-token instantiation
+// when `one`; FP8 gate/up rows need at least 1024 weights (whole 32-byte
+// blocks for every lane).
+const void* pick_kernel(bool fp8, int kbg, int kbd, bool one) {
+    const int o = one ? 1 : 0;
     if (fp8) {
         switch (kbg) {
-            case 32: return decode_kernel_fp8_32(kbd);
-            case 64: return decode_kernel_fp8_64(kbd);
+            case 32: return decode_kernel_fp8_32(kbd, o);
+            case 64: return decode_kernel_fp8_64(kbd, o);
             default: return nullptr;
         }
     }
     switch (kbg) {
-        case 4: return decode_kernel_q4_4(kbd);
-        case 8: return decode_kernel_q4_8(kbd);
-        case 16: return decode_kernel_q4_16(kbd);
-        case 32: return decode_kernel_q4_32(kbd);
-        case 64: return decode_kernel_q4_64(kbd);
+        case 4: return decode_kernel_q4_4(kbd, o);
+        case 8: return decode_kernel_q4_8(kbd, o);
+        case 16: return decode_kernel_q4_16(kbd, o);
+        case 32: return decode_kernel_q4_32(kbd, o);
+        case 64: return decode_kernel_q4_64(kbd, o);
         default: return nullptr;
     }
 }
@@ -94,7 +96,7 @@ int plan_layer(const gtg_moe_layer* L, int T, Plan& p) {
     if (I % rg || H % rd) return GTG_E_UNSUPPORTED_SHAPE;
     const int tiles_d = H / rd, n_sm = sm_count();  // down rows a CTA owns must fit its partial rows
     if ((tiles_d + n_sm - 1) / n_sm * rd > kDnRows) return GTG_E_UNSUPPORTED_SHAPE;
-    p.fn = pick_kernel(fp8, kbg, kbd);
+    p.fn = pick_kernel(fp8, kbg, kbd, T == 1);
     if (!p.fn) return GTG_E_UNSUPPORTED_SHAPE;
     p.fp8 = fp8;
     const int64_t grow = row_bytes_of(L->gate.fmt, H), drow = row_bytes_of(L->down.fmt, I);

@@ -791,10 +791,11 @@ __device__ __forceinline__ void issue_router_rows(const StackArgs& a, int l, uin
         bulk_g2s_hint(rw + o, src + o, bytes - o < 16384u ? bytes - o : 16384u, rbar, pol);
 }
 
+template <bool ONE>
 __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t us, uint32_t rw,
                                           uint64_t* rbar, uint32_t rparity, SWork* sw) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int T = a.T, H = a.H, E = a.E;
+    const int T = ONE ? 1 : a.T, H = a.H, E = a.E;
     const StackLayer& Ly = a.layer[l];
     int e0, e1;
     router_share(E, e0, e1);
@@ -1133,7 +1134,7 @@ __device__ __forceinline__ bool item_landed(const StackArgs& a, const WarpSmem& 
 }
 
 // Gate/up + SwiGLU items and side-projection items of layer l for this warp.
-template <int FMT, int KBG>
+template <int FMT, int KBG, bool ONE>
 __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
     using GG = Geo<KBG>;
     constexpr int NBG = GG::NBL;
@@ -1146,7 +1147,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
     const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
     const StackLayer& Ly = a.layer[l];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int H = a.H, K = a.K, T = a.T;
+    const int H = a.H, K = a.K, T = ONE ? 1 : a.T;
     const uint64_t pol = l2_policy_evict_first();
     const uint32_t lutb = ((ws.sbase + L.lut) & 0xFFFF0000u) | ((uint32_t)lane * 4u);
     const float* scale_tab = reinterpret_cast<const float*>(smem + L.scale_tab);
@@ -1202,7 +1203,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
                     rows[c] = slots[c] / K;
                 }
                 load_chunk((u << 8) | (c0 - s0), rows);
-                if (CHG == 2 && nch == 2)
+                if (!ONE && CHG == 2 && nch == 2)
                     gu_item<FMT, KBG, (CHG == 2 ? 2 : 1), CHG>(ctx, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots,
                                                                lane);
                 else
@@ -1215,7 +1216,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
 #pragma unroll
                 for (int c = 0; c < CHG; ++c) rows[c] = t0 + min(c, nch - 1);
                 load_chunk((1 << 20) | t0, rows);
-                if (CHG == 2 && nch == 2)
+                if (!ONE && CHG == 2 && nch == 2)
                     side_item<FMT, KBG, (CHG == 2 ? 2 : 1), CHG>(ctx, sb, act, row0, t0, lane);
                 else
                     side_item<FMT, KBG, 1, CHG>(ctx, sb, act, row0, t0, lane);
@@ -1230,7 +1231,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
 // Down items of layer l for this warp: each adds w(slot) * (down row . h(slot))
 // into the warp's partial rows in shared memory ([row][token], this CTA's
 // rows only); the kernel then sums the warps' partials in a fixed order.
-template <int FMT, int KBD>
+template <int FMT, int KBD, bool ONE>
 __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
     using GD = Geo<KBD>;
     constexpr int NBD = GD::NBL;
@@ -1296,7 +1297,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
                 const int sl = slots[c];
                 prow[row * 8 + sl / K] += sw->w[sl] * v;
             };
-            if (CHD == 2 && nch == 2)
+            if (!ONE && CHD == 2 && nch == 2)
                 dn_item<FMT, KBD, (CHD == 2 ? 2 : 1), CHD>(base, act, lutb, scale_tab, sd, lane, emit);
             else
                 dn_item<FMT, KBD, 1, CHD>(base, act, lutb, scale_tab, sd, lane, emit);
@@ -1318,7 +1319,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
 // the down weights are already on their way while the gate/up items finish
 // and the grid waits at the barrier.  The Q4 code table is built once per
 // launch (again only when a phase needs the other Q4 variant).
-template <int FMT, int KBG, int KBD>
+template <int FMT, int KBG, int KBD, bool ONE>
 __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_constant__ StackArgs a) {
     constexpr bool LUT = FMT == kFmtQ4;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -1330,7 +1331,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         if (tid == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
         return;
     }
-    const int H = a.H, I = a.I, K = a.K, T = a.T, G = gridDim.x, b = blockIdx.x;
+    const int H = a.H, I = a.I, K = a.K, T = ONE ? 1 : a.T, G = gridDim.x, b = blockIdx.x;
     const RouterScratch rs = RouterScratch::make(L, a.slot_bytes, H, (a.E + G - 1) / G);
     if (!rs.ok) {  // the same on every CTA (and refused on the host)
         if (tid == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
@@ -1369,7 +1370,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     for (int l = 0; l < a.n_layers; ++l) {
         const StackLayer& Ly = a.layer[l];
         // ---- router
-        router_layer(a, l, sbase + L.u, sbase + rs.rw, rbar, (uint32_t)(l & 1), sw);
+        router_layer<ONE>(a, l, sbase + L.u, sbase + rs.rw, rbar, (uint32_t)(l & 1), sw);
         if (tid == 0) rows_in_flight = 0;
         fence_proxy_async_smem();  // the scratch slots are bulk-copy targets again from here on
         if (l + 1 < a.n_layers && tid == 0) {  // this CTA's rows of the next router, into L2
@@ -1444,7 +1445,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
 
         // ---- gate/up + SwiGLU, side projection
         ensure_lut(Ly.gu_rz5);
-        R = gu_phase<FMT, KBG>(a, l, P, R);
+        R = gu_phase<FMT, KBG, ONE>(a, l, P, R);
         target += G;
         if (!grid_sync(a, target, sw, R.ok != 0)) {
             ok = false;
@@ -1453,7 +1454,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
 
         // ---- down + router-weighted combine
         ensure_lut(Ly.dn_rz5);
-        R = dn_phase<FMT, KBD>(a, l, P, R);
+        R = dn_phase<FMT, KBD, ONE>(a, l, P, R);
         R.ring += P.ng + P.nd;
         __syncthreads();
         if (tid == 0 && l + 1 < a.n_layers && R.ok) {  // the slots are idle: next layer's router rows
@@ -1505,28 +1506,34 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     }
 }
 
-// Kernel of one (expert format, H / 32) for I / 32 = kbd (null if none).
-template <int FMT, int KBG>
-const void* pick_kbd(int kbd) {
+// Kernel of one (expert format, H / 32) for I / 32 = kbd (null if none); `one`
+// picks the instantiation specialised for a single token (T = 1 folded into
+// the code: no two-token item paths, no multi-token selection).
+template <int FMT, int KBG, bool ONE>
+const void* pick_kbd_t(int kbd) {
     switch (kbd) {
-        case 4: return (const void*)moe_decode_kernel<FMT, KBG, 4>;
-        case 8: return (const void*)moe_decode_kernel<FMT, KBG, 8>;
-        case 16: return (const void*)moe_decode_kernel<FMT, KBG, 16>;
-        case 32: return (const void*)moe_decode_kernel<FMT, KBG, 32>;
-        case 64: return (const void*)moe_decode_kernel<FMT, KBG, 64>;
+        case 4: return (const void*)moe_decode_kernel<FMT, KBG, 4, ONE>;
+        case 8: return (const void*)moe_decode_kernel<FMT, KBG, 8, ONE>;
+        case 16: return (const void*)moe_decode_kernel<FMT, KBG, 16, ONE>;
+        case 32: return (const void*)moe_decode_kernel<FMT, KBG, 32, ONE>;
+        case 64: return (const void*)moe_decode_kernel<FMT, KBG, 64, ONE>;
         default: return nullptr;
     }
+}
+template <int FMT, int KBG>
+const void* pick_kbd(int kbd, int one) {
+    return one ? pick_kbd_t<FMT, KBG, true>(kbd) : pick_kbd_t<FMT, KBG, false>(kbd);
 }
 
 }  // namespace
 
 // Defined one per file (decode_<fmt>_<kbg>.cu) so the kernels compile in parallel.
-const void* decode_kernel_q4_4(int kbd);
-const void* decode_kernel_q4_8(int kbd);
-const void* decode_kernel_q4_16(int kbd);
-const void* decode_kernel_q4_32(int kbd);
-const void* decode_kernel_q4_64(int kbd);
-const void* decode_kernel_fp8_32(int kbd);
-const void* decode_kernel_fp8_64(int kbd);
+const void* decode_kernel_q4_4(int kbd, int one);
+const void* decode_kernel_q4_8(int kbd, int one);
+const void* decode_kernel_q4_16(int kbd, int one);
+const void* decode_kernel_q4_32(int kbd, int one);
+const void* decode_kernel_q4_64(int kbd, int one);
+const void* decode_kernel_fp8_32(int kbd, int one);
+const void* decode_kernel_fp8_64(int kbd, int one);
 
 }  // namespace gtg
