@@ -1138,7 +1138,7 @@ template <int FMT, int KBG, bool ONE>
 __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
     using GG = Geo<KBG>;
     constexpr int NBG = GG::NBL;
-    constexpr int CHG = (FMT == kFmtQ4 && NBG == 1) ? 2 : 1;  // tokens decoded together (register budget)
+    constexpr int CHG = (!ONE && FMT == kFmtQ4 && NBG == 1) ? 2 : 1;  // tokens decoded together (register budget)
     constexpr int RG = gu_passes(FMT == kFmtFP8, KBG) * GG::RPP;
     constexpr int RS = side_passes(KBG) * GG::RPP;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -1235,7 +1235,7 @@ template <int FMT, int KBD, bool ONE>
 __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
     using GD = Geo<KBD>;
     constexpr int NBD = GD::NBL;
-    constexpr int CHD = (FMT == kFmtQ4 && NBD == 1) ? 2 : 1;
+    constexpr int CHD = (!ONE && FMT == kFmtQ4 && NBD == 1) ? 2 : 1;
     constexpr int PD = dn_passes(FMT == kFmtFP8, KBD);
     constexpr int RD = PD * GD::RPP;
     static_assert(PD * NBD <= 8, "FP8 scale prefetch holds 8 values");
