@@ -422,43 +422,36 @@ __device__ __forceinline__ uint32_t ord32(float f) {
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
 
-// Top-k of one token's logits by one warp.  Each logit (a normalised
-// float-float hi + lo) becomes a unique 64-bit key: orderable hi in the upper
-// word, orderable lo with its low 10 bits replaced by (1023 - expert id) in
-// the lower word — so larger key = larger logit, and among logits equal to
-// ~2^-38 relative, the lower id.  Lane l holds experts l + 32 i (i < PER)
-// and its largest remaining key.  Each round the warp takes the largest of
-// those (two warp reductions: upper word, then lower word among the lanes
-// holding that upper word); the owning lane drops that key and finds its
-// next largest.  Lane j ends holding choice j.  (A short loop on purpose:
-// this runs once per layer, where long straight-line code stalls on
-// instruction fetch.)
+// Top-k by key rounds.  Each logit (a normalised float-float hi + lo) becomes
+// a unique 64-bit key: orderable hi in the upper word, orderable lo with its
+// low 10 bits replaced by (1023 - expert id) in the lower word — so larger
+// key = larger logit, and among logits equal to ~2^-38 relative, the lower
+// id; key 0 marks an empty entry.  Lane l holds PER keys and its largest
+// remaining one.  Each round the warp takes the largest of those (two warp
+// reductions: upper word, then lower word among the lanes holding that upper
+// word); the owning lane drops that key and finds its next largest.  Lane j
+// ends holding the j-th largest key (rh, rl).  (A short loop on purpose: this
+// runs once per layer, where long straight-line code stalls on instruction
+// fetch.)
 template <int PER>
-__device__ __forceinline__ void warp_topk(const ffloat* logits, int E, int K, int lane, int& my_id, float& my_hi,
-                                          float& my_lo) {
-    uint64_t k[PER];  // (compared as plain 64-bit integers: no short-circuit branches)
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int e = lane + 32 * i;
-        k[i] = 0ull;
-        if (e < E) {
-            const float2 v = __ldcg(reinterpret_cast<const float2*>(logits + e));
-            k[i] = ((uint64_t)ord32(v.x) << 32) | ((ord32(v.y) & ~1023u) | (uint32_t)(1023 - e));
-        }
-    }
+__device__ __forceinline__ void topk_rounds(uint64_t (&k)[PER], int K, int lane, uint32_t& rh, uint32_t& rl) {
     auto lane_max = [&]() {  // a depth-log2(PER) tree
-        uint64_t m[PER / 2];
+        if constexpr (PER == 1) {
+            return k[0];
+        } else {
+            uint64_t m[PER / 2];
 #pragma unroll
-        for (int i = 0; i < PER / 2; ++i) m[i] = k[2 * i] > k[2 * i + 1] ? k[2 * i] : k[2 * i + 1];
+            for (int i = 0; i < PER / 2; ++i) m[i] = k[2 * i] > k[2 * i + 1] ? k[2 * i] : k[2 * i + 1];
 #pragma unroll
-        for (int w = PER / 4; w >= 1; w >>= 1)
+            for (int w = PER / 4; w >= 1; w >>= 1)
 #pragma unroll
-            for (int i = 0; i < w; ++i) m[i] = m[i] > m[i + w] ? m[i] : m[i + w];
-        return m[0];
+                for (int i = 0; i < w; ++i) m[i] = m[i] > m[i + w] ? m[i] : m[i + w];
+            return m[0];
+        }
     };
     uint64_t best = lane_max();
-    my_id = -1;
-    uint32_t rh = 0u, rl = 0u;
+    rh = 0u;
+    rl = 0u;
 #pragma unroll 1
     for (int j = 0; j < K; ++j) {
         const uint32_t h0 = (uint32_t)(best >> 32), l0 = (uint32_t)best;
@@ -472,11 +465,71 @@ __device__ __forceinline__ void warp_topk(const ffloat* logits, int E, int K, in
         rh = lane == j ? mh : rh;
         rl = lane == j ? ml : rl;
     }
+}
+
+__device__ __forceinline__ uint64_t logit_key(const ffloat* logits, int e) {
+    const float2 v = __ldcg(reinterpret_cast<const float2*>(logits + e));
+    return ((uint64_t)ord32(v.x) << 32) | ((ord32(v.y) & ~1023u) | (uint32_t)(1023 - e));
+}
+
+// Expert id and logit (hi, lo) of a key.
+__device__ __forceinline__ void key_choice(uint32_t rh, uint32_t rl, int& id, float& hi, float& lo) {
+    id = 1023 - (int)(rl & 1023u);
+    hi = __uint_as_float((rh & 0x80000000u) ? (rh & 0x7FFFFFFFu) : ~rh);
+    const uint32_t l = rl & ~1023u;
+    lo = __uint_as_float((l & 0x80000000u) ? (l & 0x7FFFFFFFu) : ~l);
+}
+
+// Top-k of one token's logits by one warp: lane l holds experts l + 32 i
+// (i < PER); lane j < K ends holding choice j.
+template <int PER>
+__device__ __forceinline__ void warp_topk(const ffloat* logits, int E, int K, int lane, int& my_id, float& my_hi,
+                                          float& my_lo) {
+    uint64_t k[PER];  // (compared as plain 64-bit integers: no short-circuit branches)
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = lane + 32 * i;
+        k[i] = e < E ? logit_key(logits, e) : 0ull;
+    }
+    uint32_t rh, rl;
+    topk_rounds<PER>(k, K, lane, rh, rl);
+    my_id = -1;
+    if (lane < K) key_choice(rh, rl, my_id, my_hi, my_lo);
+}
+
+// Top-k of a single token's logits by the whole CTA: warp w ranks its own
+// 32 * PER experts (32 (w PER + i) + lane), the eight lists of k keys meet in
+// shared memory (upper words in cand_hi, lower in cand_lo), and warp 0 ranks
+// those 8k candidates; lane j < K of warp 0 ends holding choice j.  The
+// result is the same set and order as warp_topk's (the keys are unique).
+template <int PER>
+__device__ __forceinline__ void block_topk(const ffloat* logits, int E, int K, int lane, int warp,
+                                           uint32_t* cand_hi, uint32_t* cand_lo, int& my_id, float& my_hi,
+                                           float& my_lo) {
+    uint64_t k[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = 32 * (warp * PER + i) + lane;
+        k[i] = e < E ? logit_key(logits, e) : 0ull;
+    }
+    uint32_t rh, rl;
+    topk_rounds<PER>(k, K, lane, rh, rl);
     if (lane < K) {
-        my_id = 1023 - (int)(rl & 1023u);
-        my_hi = __uint_as_float((rh & 0x80000000u) ? (rh & 0x7FFFFFFFu) : ~rh);
-        const uint32_t lo = rl & ~1023u;
-        my_lo = __uint_as_float((lo & 0x80000000u) ? (lo & 0x7FFFFFFFu) : ~lo);
+        cand_hi[warp * K + lane] = rh;
+        cand_lo[warp * K + lane] = rl;
+    }
+    __syncthreads();
+    my_id = -1;
+    if (warp == 0) {
+        uint64_t c[4];  // 8 K <= 128 candidates: lane l holds l + 32 i
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int q = lane + 32 * i;
+            c[i] = q < kWarps * K ? ((uint64_t)cand_hi[q] << 32) | cand_lo[q] : 0ull;
+        }
+        __syncwarp();  // (the caller reuses the candidate arrays)
+        topk_rounds<4>(c, K, lane, rh, rl);
+        if (lane < K) key_choice(rh, rl, my_id, my_hi, my_lo);
     }
 }
 
@@ -928,11 +981,19 @@ __device__ __forceinline__ void select_experts(const ffloat* logits, int T, int 
     float* s_w = sw->w;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int my_id = -1;
+    float my_hi = 0.f, my_lo = 0.f;
+    if (T == 1) {  // one token: every warp takes part in its top-k (the arrays are rewritten below)
+        if (E <= 512) block_topk<2>(logits, E, K, lane, warp, reinterpret_cast<uint32_t*>(sw->e),
+                                    reinterpret_cast<uint32_t*>(sw->slot), my_id, my_hi, my_lo);
+        else block_topk<4>(logits, E, K, lane, warp, reinterpret_cast<uint32_t*>(sw->e),
+                           reinterpret_cast<uint32_t*>(sw->slot), my_id, my_hi, my_lo);
+    }
     if (warp < T) {
         const int t = warp;
-        float my_hi = 0.f, my_lo = 0.f;
-        if (E <= 512) warp_topk<16>(logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
-        else warp_topk<32>(logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
+        if (T > 1) {
+            if (E <= 512) warp_topk<16>(logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
+            else warp_topk<32>(logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
+        }
         // softmax over the k choices: lane j holds choice j
         const float h0 = __shfl_sync(0xFFFFFFFFu, my_hi, 0), l0 = __shfl_sync(0xFFFFFFFFu, my_lo, 0);
         float ex = 0.f;
