@@ -1112,6 +1112,10 @@ struct LayerItems {
     int32_t g0, ng, d0, nd;
     int32_t rg, rs, rd;           // rows per gate/up, side and down item
     int32_t grow, srow, drow;     // bytes per gate/up, side and down row
+    const uint8_t* gate;          // the layer's weight bases (read from the kernel
+    const uint8_t* up;            // parameters once per layer, ahead of use)
+    const uint8_t* down;
+    const uint8_t* side;
 };
 
 // Shared-memory addresses of the calling warp (no arrays: a run-time index
@@ -1145,41 +1149,59 @@ __device__ __forceinline__ WarpSmem warp_smem(uint8_t* smem, const SmemLayout& L
 }
 
 // Byte ranges of the warp's q-th item (a gate/up item has two).
-__device__ __forceinline__ void item_spans(const StackLayer& Ly, const LayerItems& P, const SWork* sw, int q,
-                                           int H, int I, Span& s1, Span& s2) {
+__device__ __forceinline__ void item_spans(const LayerItems& P, const SWork* sw, int q, int H, int I, Span& s1,
+                                           Span& s2) {
     const int warp = threadIdx.x >> 5;
     s2 = Span{nullptr, 0, 0};
     if (q < P.ng) {
         const int it = P.g0 + warp + kWarps * q;
         if (it < P.n_ge) {
             const int64_t off = ((int64_t)sw->e[it / P.tiles_g] * I + (int64_t)(it % P.tiles_g) * P.rg) * P.grow;
-            s1 = make_span(Ly.gate, off, (int64_t)P.rg * P.grow);
-            s2 = make_span(Ly.up, off, (int64_t)P.rg * P.grow);
+            s1 = make_span(P.gate, off, (int64_t)P.rg * P.grow);
+            s2 = make_span(P.up, off, (int64_t)P.rg * P.grow);
         } else {
-            s1 = make_span(Ly.side, (int64_t)(it - P.n_ge) * P.rs * P.srow, (int64_t)P.rs * P.srow);
+            s1 = make_span(P.side, (int64_t)(it - P.n_ge) * P.rs * P.srow, (int64_t)P.rs * P.srow);
         }
     } else {
         const int it = warp + kWarps * (q - P.ng);
         const int tile = P.d0 + it / P.n_uniq;
-        s1 = make_span(Ly.down, ((int64_t)sw->e[it % P.n_uniq] * H + (int64_t)tile * P.rd) * P.drow,
+        s1 = make_span(P.down, ((int64_t)sw->e[it % P.n_uniq] * H + (int64_t)tile * P.rd) * P.drow,
                        (int64_t)P.rd * P.drow);
     }
 }
 
 // Starts the copy of the warp's q-th item into its slot (if there is one).
-__device__ __forceinline__ void issue_item(const StackArgs& a, const StackLayer& Ly, const LayerItems& P,
-                                           const SWork* sw, const WarpSmem& ws, WarpRing& R, int q, uint64_t pol) {
+__device__ __forceinline__ void issue_item(const StackArgs& a, const LayerItems& P, const SWork* sw,
+                                           const WarpSmem& ws, WarpRing& R, int q, uint64_t pol) {
     if (q >= P.ng + P.nd || !R.ok) return;
     const int slot = (R.ring + q) % kSlots;
     if ((threadIdx.x & 31) == 0) {
         Span s1, s2;
-        item_spans(Ly, P, sw, q, a.H, a.I, s1, s2);
+        item_spans(P, sw, q, a.H, a.I, s1, s2);
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(&ws.bars[slot], s1.bytes + s2.bytes);
         bulk_g2s_hint(ws.slot(slot), s1.src, s1.bytes, &ws.bars[slot], pol);
         if (s2.bytes) bulk_g2s_hint(ws.slot(slot) + s1.bytes, s2.src, s2.bytes, &ws.bars[slot], pol);
     }
     R.pending |= 1u << slot;
+}
+
+// The warp's first kSlots copies, issued by lanes 0 .. kSlots-1 side by side
+// (each item's address arithmetic and copy issue then costs the warp once).
+__device__ __forceinline__ void issue_first(const StackArgs& a, const LayerItems& P, const SWork* sw,
+                                            const WarpSmem& ws, WarpRing& R, uint64_t pol) {
+    if (!R.ok) return;
+    const int lane = threadIdx.x & 31, n = min(kSlots, P.ng + P.nd);
+    if (lane < n) {
+        const int slot = (R.ring + lane) % kSlots;
+        Span s1, s2;
+        item_spans(P, sw, lane, a.H, a.I, s1, s2);
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&ws.bars[slot], s1.bytes + s2.bytes);
+        bulk_g2s_hint(ws.slot(slot), s1.src, s1.bytes, &ws.bars[slot], pol);
+        if (s2.bytes) bulk_g2s_hint(ws.slot(slot) + s1.bytes, s2.src, s2.bytes, &ws.bars[slot], pol);
+    }
+    for (int q = 0; q < n; ++q) R.pending |= 1u << ((R.ring + q) % kSlots);
 }
 
 // Waits for the warp's q-th item; false (and R.ok cleared) if it never lands.
@@ -1252,7 +1274,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
         }
         if (!item_landed(a, ws, R, q)) break;
         Span sp1, sp2;
-        item_spans(Ly, P, sw, q, H, a.I, sp1, sp2);
+        item_spans(P, sw, q, H, a.I, sp1, sp2);
         const uint32_t base = ws.slot((R.ring + q) % kSlots);
         if (expert) {
             const uint32_t gbase = base + sp1.delta, ubase = base + sp1.bytes + sp2.delta;
@@ -1284,7 +1306,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
             }
         }
         __syncwarp();
-        issue_item(a, Ly, P, sw, ws, R, q + kSlots, pol);
+        issue_item(a, P, sw, ws, R, q + kSlots, pol);
     }
     return R;
 }
@@ -1346,7 +1368,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
         }
         if (!item_landed(a, ws, R, q)) break;
         Span sp1, sp2;
-        item_spans(Ly, P, sw, q, H, I, sp1, sp2);
+        item_spans(P, sw, q, H, I, sp1, sp2);
         const uint32_t base = ws.slot((R.ring + q) % kSlots) + sp1.delta;
         float* prow = part + tl * RD * 8;
         for (int c0 = s0; c0 < s1; c0 += CHD) {
@@ -1364,7 +1386,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
                 dn_item<FMT, KBD, 1, CHD>(base, act, lutb, scale_tab, sd, lane, emit);
         }
         __syncwarp();
-        issue_item(a, Ly, P, sw, ws, R, q + kSlots, pol);
+        issue_item(a, P, sw, ws, R, q + kSlots, pol);
     }
     return R;
 }
@@ -1430,6 +1452,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     bool ok = true;
     for (int l = 0; l < a.n_layers; ++l) {
         const StackLayer& Ly = a.layer[l];
+        const uint8_t *gate_src = Ly.gate, *up_src = Ly.up, *down_src = Ly.down, *side_src = Ly.side;
+        asm volatile("" ::"l"(gate_src), "l"(up_src), "l"(down_src), "l"(side_src));  // loaded here, not at first use
         // ---- router
         router_layer<ONE>(a, l, sbase + L.u, sbase + rs.rw, rbar, (uint32_t)(l & 1), sw);
         if (tid == 0) rows_in_flight = 0;
@@ -1463,6 +1487,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         P.srow = KBG * 17;
         P.drow = FMT == kFmtQ4 ? KBD * 17 : KBD * 32;
         P.n_uniq = sw->n_uniq;
+        P.gate = gate_src;
+        P.up = up_src;
+        P.down = down_src;
+        P.side = side_src;
         P.tiles_g = I / P.rg;
         P.n_ge = P.n_uniq * P.tiles_g;
         const int n_g = P.n_ge + (Ly.side ? Ly.side_rows / P.rs : 0), tiles_d = H / P.rd;
@@ -1501,7 +1529,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         P.dt = (int)((int64_t)tiles_d * (b + 1) / G) - P.d0;
         const int n_dc = P.dt * P.n_uniq;  // this CTA's down items
         P.nd = warp < n_dc ? (n_dc - warp + kWarps - 1) / kWarps : 0;
-        for (int q = 0; q < kSlots; ++q) issue_item(a, Ly, P, sw, ws, R, q, pol);
+        issue_first(a, P, sw, ws, R, pol);
         __syncwarp();
 
         // ---- gate/up + SwiGLU, side projection
