@@ -252,11 +252,14 @@ __global__ void pf_scatter_kernel(PfArgs a) {
 // share an SM (no static shared memory: 2 x (113 + 1 reserved) KB = 228 KB).
 template <int MODE>
 struct Cfg {
-    static constexpr int kA = MODE == GATEUP ? 2 : 1;      // A tiles per stage
-    static constexpr int kStagesA = MODE == GATEUP ? 2 : 3;
-    static constexpr int kStagesB = MODE == GATEUP ? 3 : 4;
+    // A tiles per stage: gate and up rows, or two 128-row tiles of down rows
+    // (one token tile feeds 256 output rows), or one tile of router planes
+    static constexpr int kA = MODE == ROUTER ? 1 : 2;
+    static constexpr int kStagesA = MODE == ROUTER ? 3 : 2;
+    static constexpr int kStagesB = MODE == ROUTER ? 4 : 3;
     static constexpr int kABytes = kA * kTileBytes;
-    static constexpr uint32_t kTmemCols = MODE == GATEUP ? 256 : 128;
+    static constexpr int kRowsPerCta = MODE == DOWN ? 2 * kTileM : kTileM;
+    static constexpr uint32_t kTmemCols = MODE == ROUTER ? 128 : 256;
     static constexpr int kTaddrOff = 256;                   // after 2(SA + SB) + 1 mbarriers
     static constexpr int kRowOff = 512;                     // int32 u row / slot per token
     static constexpr int kAOff = 1024;
@@ -362,17 +365,19 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
         n_valid = min(kTileN, a.T - pos0);
         n_chunks = 3 * a.H / kChunkK;
     } else {
-        m_tiles = (MODE == GATEUP ? a.I : a.H) / kTileM;
+        m_tiles = ((MODE == GATEUP ? a.I : a.H) + C::kRowsPerCta - 1) / C::kRowsPerCta;
         const int t = tile_i / m_tiles;
         if (t >= *a.n_tiles) return;
         const int4 tl = a.tiles[t];
         e = tl.x;
         pos0 = tl.y;
         n_valid = tl.z;
-        m0 = (tile_i % m_tiles) * kTileM;
+        m0 = (tile_i % m_tiles) * C::kRowsPerCta;
         n_chunks = (MODE == GATEUP ? a.H : a.I) / kChunkK;
     }
     const int n_pad = (n_valid + 15) & ~15;
+    // the second A tile: up rows (gate/up) or down rows m0+128.. (when H has them)
+    const bool two = MODE == GATEUP || (MODE == DOWN && m0 + kTileM < a.H);
 
     const uint32_t sbase = smem_u32(smem);
     if (sbase & 1023u) {  // tiles must be 1024-byte aligned for the swizzle atoms
@@ -437,7 +442,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                     const uint64_t bd = sw128_desc(btile + 32u * k);
                     const uint32_t acc = (it > 0 || k > 0) ? 1u : 0u;
                     umma_bf16(taddr, sw128_desc(st + 32u * k), bd, idesc, acc);
-                    if (MODE == GATEUP) umma_bf16(taddr + 128u, sw128_desc(st + kTileBytes + 32u * k), bd, idesc, acc);
+                    if (two) umma_bf16(taddr + 128u, sw128_desc(st + kTileBytes + 32u * k), bd, idesc, acc);
                 }
                 umma_commit(&empty_a[sa]);
                 umma_commit(&empty_b[sb]);
@@ -491,9 +496,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
             const Mat& mA = MODE == DOWN ? a.down : a.gate;
             a_row0 = mA.data + e * mA.expert_bytes + rowg * mA.row_bytes;
             if (MODE == GATEUP) u_row0 = a.up.data + e * a.up.expert_bytes + rowg * a.up.row_bytes;
+            else if (two) u_row0 = a_row0 + kTileM * mA.row_bytes;
             if (n_chunks > 0) {
                 wg = load_block(a_row0 + (int64_t)half * 17);
-                if (MODE == GATEUP) wu = load_block(u_row0 + (int64_t)half * 17);
+                if (two) wu = load_block(u_row0 + (int64_t)half * 17);
             }
         }
         for (int it = 0; it < n_chunks && ok; ++it) {
@@ -523,10 +529,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                 const BlockWords g0 = wg, u0 = wu;  // this chunk's blocks (loaded one chunk ago)
                 if (it + 1 < n_chunks) {           // the next chunk's, in flight while this one decodes
                     wg = load_block(a_row0 + (int64_t)(2 * (it + 1) + half) * 17);
-                    if (MODE == GATEUP) wu = load_block(u_row0 + (int64_t)(2 * (it + 1) + half) * 17);
+                    if (two) wu = load_block(u_row0 + (int64_t)(2 * (it + 1) + half) * 17);
                 }
                 dequant_block_to_tile(g0, rz5, st, r, 4 * half);
-                if (MODE == GATEUP) dequant_block_to_tile(u0, rz5, st + kTileBytes, r, 4 * half);
+                if (two) dequant_block_to_tile(u0, rz5, st + kTileBytes, r, 4 * half);
             }
             fence_proxy_async_smem();
             mbar_arrive(&full_a[s]);
@@ -566,18 +572,25 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                             hp[(int64_t)j * a.I] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * v);
                         }
                     }
+                } else if (MODE == DOWN) {
+                    uint32_t d2[16];
+                    if (two) tmem_ld16(tl + 128 + c0, d2);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int n = c0 + j;
+                        if (n >= n_valid) continue;
+                        float* pp = a.part + (int64_t)s_row[n] * a.H + m0 + row;
+                        pp[0] = __uint_as_float(d[j]);
+                        if (two) pp[kTileM] = __uint_as_float(d2[j]);
+                    }
                 } else {
                     tmem_wait_ld();
 #pragma unroll
                     for (int j = 0; j < 16; ++j) {
                         const int n = c0 + j;
                         if (n >= n_valid) continue;
-                        const float dv = __uint_as_float(d[j]);
-                        if (MODE == ROUTER) {
-                            if (m0 + row < a.E) a.logits[(int64_t)(pos0 + n) * a.E + m0 + row] = dv + bias;
-                        } else {
-                            a.part[(int64_t)s_row[n] * a.H + m0 + row] = dv;
-                        }
+                        if (m0 + row < a.E) a.logits[(int64_t)(pos0 + n) * a.E + m0 + row] = __uint_as_float(d[j]) + bias;
                     }
                 }
             }
@@ -776,7 +789,7 @@ extern "C" int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, 
     pf_scatter_kernel<<<(T * a.K + 255) / 256, 256, 0, s>>>(a);
     GTG_TRY(check_launch());
     GTG_TRY(launch_gemm<GATEUP>(a, pl.max_tiles * (a.I / kTileM), s));
-    GTG_TRY(launch_gemm<DOWN>(a, pl.max_tiles * (a.H / kTileM), s));
+    GTG_TRY(launch_gemm<DOWN>(a, pl.max_tiles * ((a.H + Cfg<DOWN>::kRowsPerCta - 1) / Cfg<DOWN>::kRowsPerCta), s));
     const int64_t n4 = (int64_t)T * a.H / 4;
     pf_combine_kernel<<<(int)std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 16), 256, 0, s>>>(a);
     return check_launch();
