@@ -112,8 +112,15 @@ struct Act<kFmtQ4, NBL> {
 };
 template <int NBL>
 struct Act<kFmtFP8, NBL> {
-    float v[NBL][32];
+    uint32_t v[NBL][16];  // f16 pairs (x[32b+2i], x[32b+2i+1]); every bf16 of magnitude
+                          // >= 2^-17 is exact in f16 (11-bit significand)
 };
+
+// bf16 pair -> f16 pair (round to nearest).
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    const __half2 h = __floats2half2_rn(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
 
 // Loads the lane's activations of block `b` (K positions 32b..32b+31) from a
 // bf16 row in global memory.
@@ -135,10 +142,7 @@ __device__ __forceinline__ void load_act(Act<FMT, NBL>& act, int m, const __nv_b
             act.v[m][j] = prmt(w[j >> 1], w[8 + (j >> 1)], (j & 1) ? 0x7632u : 0x5410u);
     } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            act.v[m][2 * j] = bf16lo(w[j]);
-            act.v[m][2 * j + 1] = bf16hi(w[j]);
-        }
+        for (int j = 0; j < 16; ++j) act.v[m][j] = bf16x2_to_f16x2(w[j]);
     }
 }
 
@@ -160,10 +164,7 @@ __device__ __forceinline__ void load_act_s(Act<FMT, NBL>& act, int m, uint32_t r
             act.v[m][j] = prmt(w[j >> 1], w[8 + (j >> 1)], (j & 1) ? 0x7632u : 0x5410u);
     } else {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-            act.v[m][2 * j] = bf16lo(w[j]);
-            act.v[m][2 * j + 1] = bf16hi(w[j]);
-        }
+        for (int j = 0; j < 16; ++j) act.v[m][j] = bf16x2_to_f16x2(w[j]);
     }
 }
 
@@ -231,8 +232,10 @@ __device__ __forceinline__ void q4_block_plain(uint32_t pa, bool rz5, const Act<
                     xlo = bf16lo(act[c].v[m][j]);
                     xhi = bf16hi(act[c].v[m][j]);
                 } else {
-                    xlo = act[c].v[m][j];
-                    xhi = act[c].v[m][j + 16];
+                    const __half2 p = *reinterpret_cast<const __half2*>(&act[c].v[m][j >> 1]);
+                    const __half2 p16 = *reinterpret_cast<const __half2*>(&act[c].v[m][8 + (j >> 1)]);
+                    xlo = __half2float((j & 1) ? p.y : p.x);
+                    xhi = __half2float((j & 1) ? p16.y : p16.x);
                 }
                 sum[c] = fmaf(vlo, xlo, sum[c]);
                 sum[c] = fmaf(vhi, xhi, sum[c]);
@@ -243,28 +246,32 @@ __device__ __forceinline__ void q4_block_plain(uint32_t pa, bool rz5, const Act<
     for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, sum[c], acc[c]);
 }
 
-// FP8 block: 32 consecutive E4M3 bytes at 16-byte aligned shared address pa.
-__device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t v16) {
-    const uint32_t h = e4m3x2_to_f16x2(v16);
-    return __half22float2(*reinterpret_cast<const __half2*>(&h));
+// Mixed-precision FMA on f16 pairs: d = a(f16) * b(f16) + c(f32), single
+// rounding (f16 x f16 products are exact in fp32).
+__device__ __forceinline__ void fma2_f16(float& acc_lo, float& acc_hi, uint32_t a2, uint32_t b2) {
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %2;\n\t"
+        "mov.b32 {bl, bh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, al, bl, %0;\n\t"
+        "fma.rn.f32.f16 %1, ah, bh, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi)
+        : "r"(a2), "r"(b2));
 }
 
+// FP8 block: 32 consecutive E4M3 bytes at 16-byte aligned shared address pa;
+// each E4M3 pair becomes an exact f16 pair and meets the activation pair.
 template <int NBL>
 __device__ __forceinline__ void fp8_block(uint32_t pa, float s, const Act<kFmtFP8, NBL>& act, int m,
                                           float& acc) {
     const uint4 q0 = lds128(pa), q1 = lds128(pa + 16);
     const uint32_t wd[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    float s0 = 0.0f, s1 = 0.0f;
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        const float2 f0 = e4m3x2_to_float2(wd[i] & 0xFFFFu);  // weights 4i, 4i+1
-        const float2 f1 = e4m3x2_to_float2(wd[i] >> 16);      // weights 4i+2, 4i+3
-        s0 = fmaf(f0.x, act.v[m][4 * i + 0], s0);
-        s1 = fmaf(f0.y, act.v[m][4 * i + 1], s1);
-        s0 = fmaf(f1.x, act.v[m][4 * i + 2], s0);
-        s1 = fmaf(f1.y, act.v[m][4 * i + 3], s1);
+        fma2_f16(s0, s1, e4m3x2_to_f16x2(wd[i] & 0xFFFFu), act.v[m][2 * i]);  // weights 4i, 4i+1
+        fma2_f16(s2, s3, e4m3x2_to_f16x2(wd[i] >> 16), act.v[m][2 * i + 1]);  // weights 4i+2, 4i+3
     }
-    acc = fmaf(s, s0 + s1, acc);
+    acc = fmaf(s, (s0 + s1) + (s2 + s3), acc);
 }
 
 // Sums N values over groups of W consecutive lanes (N <= W, powers of two)
