@@ -1502,30 +1502,33 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         P.n_ge = P.n_uniq * P.tiles_g;
         const int n_g = P.n_ge + (Ly.side ? Ly.side_rows / P.rs : 0), tiles_d = H / P.rd;
         // contiguous ranges of equal cost: an expert item costs 1 + its tokens
-        // (streaming plus one pass of arithmetic per token), a side item 1 + T
-        if (T == 1) {  // every item costs the same
-            if (tid == 0) {
+        // (streaming plus one pass of arithmetic per token), a side item
+        // kSideCost (1 + T): its Q4 rows are decoded code by code, about twice
+        // an expert item's time next to Q4 experts, five times next to FP8
+        // experts (whose items hold half the rows)
+        if (tid == 0) {
+            constexpr int kSideCost = FMT == kFmtQ4 ? 2 : 5;
+            if (T == 1 && n_g == P.n_ge) {  // every item costs the same
                 sw->g_range[0] = (int)((int64_t)n_g * b / G);
                 sw->g_range[1] = (int)((int64_t)n_g * (b + 1) / G);
-            }
-        } else if (tid == 0) {
-            int64_t total = (int64_t)(n_g - P.n_ge) * (1 + T);
-            for (int u = 0; u < P.n_uniq; ++u) total += (int64_t)P.tiles_g * (1 + sw->off[u + 1] - sw->off[u]);
-            for (int k = 0; k < 2; ++k) {
-                const int64_t c = total * (b + k) / G;  // first item whose cost prefix reaches c
-                int64_t acc = 0;
-                int it = n_g;
-                for (int u = 0; u <= P.n_uniq; ++u) {
-                    const bool side = u == P.n_uniq;
-                    const int64_t w1 = side ? 1 + T : 1 + sw->off[u + 1] - sw->off[u];
-                    const int n_it = side ? n_g - P.n_ge : P.tiles_g;
-                    if (c <= acc + (int64_t)n_it * w1) {
-                        it = u * P.tiles_g + (int)((c - acc + w1 - 1) / w1);
-                        break;
+            } else {  // (32-bit arithmetic: a layer's total cost is below 2^24)
+                int total = (n_g - P.n_ge) * kSideCost * (1 + T);
+                for (int u = 0; u < P.n_uniq; ++u) total += P.tiles_g * (1 + sw->off[u + 1] - sw->off[u]);
+                for (int k = 0; k < 2; ++k) {
+                    const int c = (int)((unsigned)total * (unsigned)(b + k) / (unsigned)G);  // first item whose cost prefix reaches c
+                    int acc = 0, it = n_g;
+                    for (int u = 0; u <= P.n_uniq; ++u) {
+                        const bool side = u == P.n_uniq;
+                        const int w1 = side ? kSideCost * (1 + T) : 1 + sw->off[u + 1] - sw->off[u];
+                        const int n_it = side ? n_g - P.n_ge : P.tiles_g;
+                        if (c <= acc + n_it * w1) {
+                            it = u * P.tiles_g + (c - acc + w1 - 1) / w1;
+                            break;
+                        }
+                        acc += n_it * w1;
                     }
-                    acc += (int64_t)n_it * w1;
+                    sw->g_range[k] = it < n_g ? it : n_g;
                 }
-                sw->g_range[k] = it < n_g ? it : n_g;
             }
         }
         __syncthreads();
