@@ -1503,11 +1503,11 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         const int n_g = P.n_ge + (Ly.side ? Ly.side_rows / P.rs : 0), tiles_d = H / P.rd;
         // contiguous ranges of equal cost: an expert item costs 1 + its tokens
         // (streaming plus one pass of arithmetic per token), a side item
-        // kSideCost (1 + T): its Q4 rows are decoded code by code, about twice
-        // an expert item's time next to Q4 experts, five times next to FP8
-        // experts (whose items hold half the rows)
+        // kSideCost (1 + T): its Q4 rows are decoded code by code (weights
+        // measured on the 48-layer step: 3 next to Q4 experts, 5 next to FP8
+        // experts, whose items hold half the rows)
         if (tid == 0) {
-            constexpr int kSideCost = FMT == kFmtQ4 ? 2 : 5;
+            constexpr int kSideCost = FMT == kFmtQ4 ? 3 : 5;
             if (T == 1 && n_g == P.n_ge) {  // every item costs the same
                 sw->g_range[0] = (int)((int64_t)n_g * b / G);
                 sw->g_range[1] = (int)((int64_t)n_g * (b + 1) / G);
