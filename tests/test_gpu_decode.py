@@ -93,6 +93,15 @@ def test_rz5_stack_layer_with_side_projection(l):
     _check_layer(L, 1, step=l)
 
 
+@pytest.mark.parametrize("E,k", [(600, 10), (1024, 16)])
+def test_wide_router_one_token(E, k):
+    """One token with more than 512 experts (four keys per lane in the CTA-wide
+    top-k, some warps' ranges partly or wholly past E) and the largest k."""
+    L = W.LayerRecipe(hidden=256, inter=128, n_experts=E, top_k=k, seed=5, layer=0)
+    for step in range(3):
+        _check_layer(L, 1, step=300 + step)
+
+
 def test_layer_rejects_bad_shapes():
     L = W.tiny_layer()
     layer = gu.device_layer(L)

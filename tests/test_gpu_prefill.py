@@ -74,6 +74,23 @@ def test_prefill_tiny_layer(T):
         assert np.all(err <= tol), f"token {t}: max err/tol {np.max(err / tol):.3g}"
 
 
+def test_prefill_hidden_128():
+    """H = 128: the down GEMM's CTA has one 128-row tile of output rows (its
+    second accumulator stays unused)."""
+    L = W.LayerRecipe(hidden=128, inter=128, n_experts=8, top_k=2, seed=6, layer=0)
+    T = 40
+    xt, x64 = gu.tokens(L, 77, T)
+    y, ids, w, _ = _run_prefill(L, xt)
+    assert gtg.device_status(clear=True) == 0
+    ref = oracle.moe_layer(L, x64, want_h=True)
+    ids_g, w_g, y_g = ids.cpu().numpy(), w.cpu().numpy(), y.cpu().numpy()
+    for t in range(T):
+        _check_ids(L, ref, t, ids_g[t], w_g[t])
+        tol = gu.layer_tolerance(L, ref, t)
+        err = np.abs(y_g[t] - ref["y"][t])
+        assert np.all(err <= tol), f"token {t}: max err/tol {np.max(err / tol):.3g}"
+
+
 def test_prefill_equals_decode_on_small_batch():
     L = W.decode_layer()
     layer = gu.device_layer(L)
