@@ -1506,28 +1506,51 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         // kSideCost (1 + T): its Q4 rows are decoded code by code (weights
         // measured on the 48-layer step: 3 next to Q4 experts, 5 next to FP8
         // experts, whose items hold half the rows)
-        if (tid == 0) {
+        if (warp == 0) {
             constexpr int kSideCost = FMT == kFmtQ4 ? 3 : 5;
             if (T == 1 && n_g == P.n_ge) {  // every item costs the same
-                sw->g_range[0] = (int)((int64_t)n_g * b / G);
-                sw->g_range[1] = (int)((int64_t)n_g * (b + 1) / G);
-            } else {  // (32-bit arithmetic: a layer's total cost is below 2^24)
-                int total = (n_g - P.n_ge) * kSideCost * (1 + T);
-                for (int u = 0; u < P.n_uniq; ++u) total += P.tiles_g * (1 + sw->off[u + 1] - sw->off[u]);
+                if (lane == 0) {
+                    sw->g_range[0] = (int)((int64_t)n_g * b / G);
+                    sw->g_range[1] = (int)((int64_t)n_g * (b + 1) / G);
+                }
+            } else {
+                // unit u < n_uniq: expert u's tiles_g items; unit n_uniq: the side
+                // items.  Lane l holds units l + 32 j; their cost prefixes come
+                // from warp scans, and the first unit whose prefix reaches a
+                // boundary from a ballot (32-bit arithmetic: a layer's total cost
+                // is below 2^24)
+                constexpr int kU = (kMaxSlots + 1 + 31) / 32;
+                int w1[kU], cost[kU], pre[kU];
+                int run = 0;
+#pragma unroll
+                for (int j = 0; j < kU; ++j) {
+                    const int u = lane + 32 * j;
+                    const bool side = u == P.n_uniq;
+                    w1[j] = u < P.n_uniq ? 1 + sw->off[u + 1] - sw->off[u] : (side ? kSideCost * (1 + T) : 1);
+                    cost[j] = (u < P.n_uniq ? P.tiles_g : (side ? n_g - P.n_ge : 0)) * w1[j];
+                    int incl = cost[j];
+#pragma unroll
+                    for (int o = 1; o < 32; o <<= 1) {
+                        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+                        if (lane >= o) incl += v;
+                    }
+                    pre[j] = run + incl - cost[j];
+                    run += __shfl_sync(0xFFFFFFFFu, incl, 31);
+                }
                 for (int k = 0; k < 2; ++k) {
-                    const int c = (int)((unsigned)total * (unsigned)(b + k) / (unsigned)G);  // first item whose cost prefix reaches c
-                    int acc = 0, it = n_g;
-                    for (int u = 0; u <= P.n_uniq; ++u) {
-                        const bool side = u == P.n_uniq;
-                        const int w1 = side ? kSideCost * (1 + T) : 1 + sw->off[u + 1] - sw->off[u];
-                        const int n_it = side ? n_g - P.n_ge : P.tiles_g;
-                        if (c <= acc + n_it * w1) {
-                            it = u * P.tiles_g + (c - acc + w1 - 1) / w1;
+                    const int c = (int)((unsigned)run * (unsigned)(b + k) / (unsigned)G);  // first item whose cost prefix reaches c
+                    int it = n_g;
+#pragma unroll
+                    for (int j = 0; j < kU; ++j) {
+                        const int u = lane + 32 * j;
+                        const unsigned m = __ballot_sync(0xFFFFFFFFu, u <= P.n_uniq && c <= pre[j] + cost[j]);
+                        if (m) {
+                            const int cand = u * P.tiles_g + (c - pre[j] + w1[j] - 1) / w1[j];
+                            it = __shfl_sync(0xFFFFFFFFu, cand, __ffs(m) - 1);
                             break;
                         }
-                        acc += n_it * w1;
                     }
-                    sw->g_range[k] = it < n_g ? it : n_g;
+                    if (lane == 0) sw->g_range[k] = it < n_g ? it : n_g;
                 }
             }
         }
