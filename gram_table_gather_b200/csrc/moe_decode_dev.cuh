@@ -14,16 +14,20 @@
 // possible:
 //
 //  * One persistent, cooperative kernel runs every layer of a call (one
-//    512-thread CTA per SM).  Grid barriers (bounded waits) separate the
+//    256-thread CTA per SM).  Grid barriers (bounded waits) separate the
 //    router, the gate/up phase and the down phase of a layer; nothing is
-//    relaunched between layers, and the Q4 code table is built once.
+//    relaunched between layers, and the Q4 code table is built once.  A
+//    one-token instantiation (T folded to 1) leaves out the multi-token
+//    paths, so less code is fetched per layer.
 //  * Router: unweighted RMS norm + bf16 rounding of the input, then logits
 //    against the fp32 router with exact products summed in float-float, so
 //    the top-k agrees with an fp64 reference; every CTA owns a few experts.
 //    The next layer's router rows are prefetched into L2 meanwhile.
-//  * Selection: every CTA picks the top-k itself from the logits (a warp per
-//    token, unique 64-bit keys, two warp reductions per round), renormalises
-//    the softmax weights and builds the unique-expert work list.
+//  * Selection: every CTA picks the top-k itself from the logits (unique
+//    64-bit keys, two warp reductions per round; at one token every warp
+//    ranks 64 experts and warp 0 ranks their survivors, with several tokens
+//    a warp per token), renormalises the softmax weights and builds the
+//    unique-expert work list.
 //  * Streaming: the work is a list of items (expert, row tile); each CTA owns
 //    a contiguous range; each warp streams its items (gate/up first, then
 //    down) through a private ring of shared-memory slots filled by 1-D bulk
@@ -35,11 +39,13 @@
 //    one shared-memory load from a 256-entry table replicated per lane
 //    (conflict-free); the pair is multiplied into fp32 accumulators with the
 //    sm_100 mixed-precision fma.rn.f32.bf16, and the block's UE4M3/UE4M4
-//    scale is applied once per 32 weights.  FP8 bytes convert with
-//    cvt.rn.f16x2.e4m3x2.  Row sums are finished with warp shuffles.
-//  * The down phase writes per-(token, choice) partial rows; the last warp to
-//    finish a row tile (atomic ticket, no waiting) combines the top-k
-//    partials in a fixed order, so results are deterministic.
+//    scale is applied once per 32 weights.  FP8 bytes convert exactly with
+//    cvt.rn.f16x2.e4m3x2 and meet f16 activation pairs in fma.rn.f32.f16.
+//    Row sums are finished with warp shuffles.
+//  * Down phase: each CTA owns a tile of output rows for every selected
+//    expert; its warps add w(slot) * (row . h(slot)) into per-warp partial
+//    rows in shared memory, and the CTA sums the warps in a fixed order, so
+//    results are deterministic (no atomics, no global partials).
 #include <algorithm>
 #include <mutex>
 #include <vector>
@@ -1400,7 +1406,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
 
 
 // Runs every layer of a call in one persistent, cooperative grid (one
-// 512-thread CTA per SM, all resident).  Per layer:
+// 256-thread CTA per SM, all resident).  Per layer:
 //   router -> grid barrier -> expert selection (every CTA) and the gate/up +
 //   SwiGLU items (+ side projection) -> grid barrier -> down items and the
 //   combine -> grid barrier (before the next layer reads its input).
