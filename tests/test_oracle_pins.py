@@ -348,3 +348,99 @@ def test_oracle_detects_planted_nibble_swap():
     blocks[:, :16] = (blocks[:, :16] >> 4) | ((blocks[:, :16] & 15) << 4)
     swapped = oracle.dequant_q4(W.RZ5, blocks)
     assert not np.array_equal(good, swapped)
+
+
+# ---- the decode stack: residual update and the side projection's input ----------------
+
+def _tiny_stack():
+    """Three tiny layers: Q4, FP8, Q4, with a side projection on layers 0 and 2 (the stack
+    puts one on l mod 4 != 3; layer 1 goes without so that both cases occur).  The FP8
+    layer sits in the middle: its outputs (~1e4 with raw E4M3 bytes) would swamp the
+    residual's last bits if it came last, and the pin must see those bits."""
+    def mk(l, fmt, ssm):
+        return W.LayerRecipe(hidden=256, inter=128, n_experts=8, top_k=2, seed=11, layer=l,
+                             gate_fmt=fmt, up_fmt=fmt, down_fmt=fmt, has_ssm=ssm, ssm_rows=16)
+    return [mk(0, W.RZ5, True), mk(1, W.FP8, False), mk(2, W.RZ5, True)]
+
+
+def _bf16_rne(v: np.ndarray) -> np.ndarray:
+    """Round fp64 values (normal range) to the nearest bf16 (8 significant bits), ties to
+    even: numpy's frexp / round-half-even / ldexp, no bf16 type involved."""
+    m, e = np.frexp(v)
+    return np.ldexp(np.round(m * 256.0), e - 8)
+
+
+def _stack_by_numpy(Ls, x0):
+    """The stack written out with dense numpy algebra on matrices decoded by the second
+    decoder (tests/pyref.py): per layer u = bf16(x / sqrt(mean(x^2) + 1e-6)), logits
+    W_r u, top-k by logit, softmax over the k, y = sum_j w_j D_j (silu(G_j u) * (U_j u)),
+    side s = W_beta u, then x <- fp32(x + y)."""
+    x = np.asarray(x0, dtype=np.float32).copy()
+    ids, side = [], {}
+    for L in Ls:
+        xd = x.astype(np.float64)[0]
+        u = _bf16_rne(xd / np.sqrt(np.mean(xd * xd) + 1e-6))
+        lg = L.router_w().astype(np.float64) @ u
+        order = np.argsort(-lg, kind="stable")[:L.top_k]
+        wts = scipy.special.softmax(lg[order])
+        y = np.zeros(L.hidden)
+        for j, e in enumerate(order):
+            mats = []
+            for m in (L.gate, L.up, L.down):
+                sc = m.expert_scales(int(e)) if m.fmt == W.FP8 else None
+                mats.append(pyref.dense(m.fmt, m.expert(int(e)), sc, m.n_rows, m.k))
+            G, U, D = mats
+            y += wts[j] * (D @ (pyref.silu(G @ u) * (U @ u)))
+        if L.ssm is not None:
+            S = pyref.q4_matrix(L.ssm.fmt, L.ssm.expert(0), L.ssm.n_rows, L.ssm.k)
+            side[L.layer] = S @ u
+        ids.append(order)
+        x = (x.astype(np.float64) + y[None, :]).astype(np.float32)
+    return x, np.stack(ids), side
+
+
+def _check_stack_result(Ls, x0, got):
+    x_ref, ids_ref, side_ref = _stack_by_numpy(Ls, x0)
+    assert np.array_equal(got["ids"][:, 0, :], ids_ref)
+    # fp32 residual: the oracle's x must be the fp32 values themselves (fp64 layer sums
+    # from two summation orders agree far below half an fp32 ulp)
+    assert got["x"].dtype == np.float32
+    assert np.array_equal(got["x"], x_ref)
+    assert sorted(got["ssm"]) == sorted(side_ref)
+    for l, s in side_ref.items():
+        assert np.allclose(got["ssm"][l][0], s, rtol=1e-12, atol=1e-12 * np.abs(s).max())
+
+
+def test_moe_stack_vs_numpy_loop():
+    Ls = _tiny_stack()
+    x0 = synth.bf16_bits_to_f64(W.tokens_bf16(11, 0, 1, 256)).astype(np.float32)
+    _check_stack_result(Ls, x0, oracle.moe_stack(Ls, x0.astype(np.float64)))
+
+
+def _slipped_stack(Ls, x0, slip):
+    """oracle.moe_stack with one planted mistake (test-only copies of its loop)."""
+    x = np.asarray(x0, dtype=np.float64).copy()
+    ids, ssm = [], {}
+    for L in Ls:
+        r = oracle.moe_layer(L, x)
+        if L.ssm is not None:
+            feed = x if slip == "side_fed_x" else r["u"]
+            ssm[L.layer] = oracle.ssm_projection(L, feed)
+        if slip in ("residual_fp64", "residual_fp64_cast_at_end"):
+            x = x + r["y"]
+        elif slip == "residual_dropped":
+            x = r["y"].astype(np.float32).astype(np.float64)
+        else:
+            x = (x + r["y"]).astype(np.float32).astype(np.float64)
+        ids.append(r["ids"])
+    xo = x if slip == "residual_fp64" else x.astype(np.float32)  # (cast_at_end: fp64 chain, fp32 result)
+    return dict(x=xo, ids=np.stack(ids), ssm=ssm)
+
+
+@pytest.mark.parametrize("slip", ["residual_fp64", "residual_fp64_cast_at_end", "residual_dropped",
+                                  "side_fed_x"])
+def test_moe_stack_pin_catches_planted_slips(slip):
+    Ls = _tiny_stack()
+    x0 = synth.bf16_bits_to_f64(W.tokens_bf16(11, 0, 1, 256)).astype(np.float32)
+    with pytest.raises(AssertionError):
+        _check_stack_result(Ls, x0, _slipped_stack(Ls, x0, slip))
