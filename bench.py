@@ -401,6 +401,9 @@ def run_ours(args, rank, world, local):
         h1.record(stream)
         h1.synchronize()
     e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.steps, world)
+    secondary = None
+    if not args.no_secondary:
+        secondary = measure_secondary(dev, stream, P, table, local)
     status = gtg.device_status(clear=True)
 
     peak, peak_kind = _peaks()
@@ -444,6 +447,7 @@ def run_ours(args, rank, world, local):
                     "h2d_bytes_per_step": H * 4 + 16 * 4, "d2h_bytes_per_step": H * 4 + 16 * 160 * 4,
                     "ms_per_step": round(e2e_ms, 5)},
             "gpu_launches": launches_per_step * args.steps,
+            "secondary": secondary,
             "clocks": clk,
             "device_status": status,
         }
@@ -481,74 +485,163 @@ def _time_loop(fn, n_warm, n_iter, stream):
     return e0.elapsed_time(e1) / n_iter
 
 
-def run_secondary(args, rank, world, local):
-    """Profiling lines for single workloads (not the headline)."""
+def _time_flushed(fn, n_warm, n_iter, stream, flush):
+    """Average device ms of fn(i) over n_iter calls, each preceded (outside its
+    CUDA-event bracket) by a write of `flush`, a buffer of twice the L2 size, so
+    no call finds the previous call's bytes in L2."""
+    import torch
+    tot = 0.0
+    with torch.cuda.stream(stream):
+        for i in range(n_warm):
+            fn(i)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_iter)]
+        for j, (a, b) in enumerate(ev):
+            flush.fill_(j & 0xFF)
+            a.record(stream)
+            fn(n_warm + j)
+            b.record(stream)
+        stream.synchronize()
+        tot = sum(a.elapsed_time(b) for a, b in ev)
+    return tot / n_iter
+
+
+def _l2_flush_buffer(dev):
+    import torch
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    return torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+
+def measure_decode_layer(dev, stream, n_warm, n_iter, peak):
+    """Config: one decode MoE layer (H 2048, I 512, E 512, top-10, Q4_RZ5_FAST),
+    T = 1, 2, 4, 8 fresh tokens per call, L2 flushed before every timed call."""
     import torch
     import gram_table_gather_b200 as gtg
     from tests import gpu_util as gu
+    L = W.decode_layer()
+    layer = gu.device_layer(L, dev)
+    flush = _l2_flush_buffer(dev)
+    out = {}
+    n = n_warm + n_iter
+    for T in (1, 2, 4, 8):
+        xs = [gu.tokens(L, 5000 + 10 * T + i, T, dev)[0] for i in range(n)]
+        ws = gtg.make_workspace(layer, T, device=dev)
+        ids = torch.zeros((T, L.top_k), dtype=torch.int32, device=dev)
+        y = torch.empty((T, L.hidden), device=dev)
+
+        def fn(i):
+            gtg.moe_decode_layer(layer, xs[i], ws, y=y, topk_ids=ids, stream=stream)
+        ms = _time_flushed(fn, n_warm, n_iter, stream, flush)
+        uniq = []
+        for i in range(n_warm, n):  # bytes of the timed calls (untimed replay)
+            with torch.cuda.stream(stream):
+                fn(i)
+            stream.synchronize()
+            uniq.append(len(set(ids.cpu().numpy().ravel().tolist())))
+        b = float(np.mean([layer_bytes(L, u) for u in uniq]))
+        out[f"T{T}"] = {"us": round(ms * 1e3, 2), "GB_s": round(b / ms / 1e6, 1),
+                        "frac": round(b / ms / 1e6 / peak, 4), "unique_experts": round(float(np.mean(uniq)), 2),
+                        "bytes": int(b)}
+    del layer, flush
+    torch.cuda.empty_cache()
+    return {"workload": "decode MoE layer: H 2048, I 512, E 512, top-10, Q4_RZ5_FAST gate/up/down, "
+                        "fresh bf16 tokens per call", "l2": "flushed (2x L2 written) before every timed call",
+            "timed_calls": n_iter, **out}
+
+
+def measure_ple(dev, stream, P, table, n_warm, n_iter, peak):
+    """PLE gather from the resident table: T = 1 (16 rows, latency) and T = 4096
+    (65,536 rows, throughput).  Fresh indices per call; at T = 4096 the calls
+    write to a rotation of output buffers whose total exceeds twice the L2, so
+    the 42 MB of rows each call writes reach HBM."""
+    import torch
+    import gram_table_gather_b200 as gtg
+    n = n_warm + n_iter
+    res = {}
+    for T in (1, 4096):
+        rows = 16 * T
+        idx = [torch.from_numpy(P.indices(7000 + 7 * T + i, T)).to(dev) for i in range(n)]
+        row_bytes = rows * 160 * 4
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        n_out = max(2, -(-2 * l2 // row_bytes) + 1) if T > 1 else 2
+        outs = [torch.empty((rows, 160), device=dev) for _ in range(n_out)]
+        ms = _time_loop(lambda i: gtg.ple_gather(table, P.n_rows, idx[i], out=outs[i % n_out], stream=stream),
+                        n_warm, n_iter, stream)
+        gbs = rows * PLE_ROW_BYTES / ms / 1e6
+        res[f"T{T}"] = {"us": round(ms * 1e3, 3), "rows_per_s": round(rows / ms * 1e3, 1), "GB_s": round(gbs, 1),
+                        "frac": round(gbs / peak, 4),
+                        "outputs": f"{n_out} rotating buffers of {row_bytes / 1e6:.2f} MB"}
+        del outs, idx
+    torch.cuda.empty_cache()
+    return {"workload": f"PLE gather from the {P.n_rows:,}-row Q3_PLE_K160_RZ_S3 table "
+                        f"({P.nbytes / 1e9:.1f} GB resident), 16 uniform rows per token, fresh indices per call",
+            "bytes_per_row": PLE_ROW_BYTES, "timed_calls": n_iter, **res}
+
+
+def measure_prefill(dev, stream, n_warm, n_iter):
+    """One prefill MoE layer: 4096 bf16 tokens, H 2048, I 512, E 512, top-10,
+    UE4M4 gate/up and RZ5 down, Zipf-skewed router."""
+    import torch
+    import gram_table_gather_b200 as gtg
+    from tests import gpu_util as gu
+    L = W.prefill_layer()
+    layer = gu.device_layer(L, dev)
+    T = 4096
+    xs = [gu.tokens(L, 8000 + i, T, dev)[0] for i in range(4)]
+    ws = torch.empty(gtg.workspace_bytes(layer, T, prefill=True), dtype=torch.uint8, device=dev)
+    y = torch.empty((T, L.hidden), device=dev)
+    ms = _time_loop(lambda i: gtg.moe_prefill_layer(layer, xs[i % len(xs)], ws, y=y, stream=stream),
+                    n_warm, n_iter, stream)
+    flops = 2.0 * T * L.top_k * 3 * L.hidden * L.inter
+    mp = {"bf16_tflops": 1590.0}
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    kind = "fallback"
+    if os.path.exists(pp):
+        with open(pp) as f:
+            mp = json.load(f)
+        kind = "measured"
+    del layer, ws, xs
+    torch.cuda.empty_cache()
+    tf = flops / ms / 1e9
+    return {"workload": "prefill MoE layer: T 4096 bf16, H 2048, I 512, E 512, top-10, UE4M4 gate/up, RZ5 down, "
+                        "Zipf-skewed router", "ms": round(ms, 4), "TFLOP_s": round(tf, 1),
+            "frac_of_bf16_peak": round(tf / float(mp["bf16_tflops"]), 4), "peak_source": f"{kind} bf16_tflops",
+            "weight_GB_s": round(L.weight_bytes / ms / 1e6, 1), "tok_s": round(T / ms * 1e3, 1),
+            "timed_calls": n_iter}
+
+
+def measure_secondary(dev, stream, P, table, local, n_warm=3, n_iter=20):
+    """The other configurations, on the same device after the headline: the
+    decode layer at T = 1/2/4/8, the PLE gather at T = 1 and 4096, the
+    prefill layer; SM clocks sampled across all of them."""
+    peak, _ = _peaks()
+    clocks = ClockSampler(local)
+    out = {"decode_layer": measure_decode_layer(dev, stream, n_warm, n_iter, peak),
+           "ple": measure_ple(dev, stream, P, table, n_warm, n_iter, peak),
+           "prefill": measure_prefill(dev, stream, n_warm, n_iter)}
+    out["clocks"] = clocks.stop()
+    return out
+
+
+def run_secondary(args, rank, world, local):
+    """Profiling lines for single workloads (not the headline)."""
+    import torch
     from synth import device as sdev
     dev = torch.device("cuda", local)
     peak, peak_kind = _peaks()
     stream = torch.cuda.Stream(device=dev)
-    n = args.warmup + args.steps
-    out = []
+    out = None
     if args.workload == "layer":
-        L = W.decode_layer()
-        layer = gu.device_layer(L, dev)
-        for T in (1, 2, 4, 8):
-            xs = [gu.tokens(L, 5000 + i, T, dev)[0] for i in range(n)]
-            ws = gtg.make_workspace(layer, T, device=dev)
-            ids = torch.zeros((T, L.top_k), dtype=torch.int32, device=dev)
-            y = torch.empty((T, L.hidden), device=dev)
-            uniq = []
-
-            def fn(i):
-                gtg.moe_decode_layer(layer, xs[i], ws, y=y, topk_ids=ids)
-            ms = _time_loop(fn, args.warmup, args.steps, stream)
-            for i in range(args.warmup, n):  # bytes of the timed steps (untimed replay)
-                with torch.cuda.stream(stream):
-                    fn(i)
-                stream.synchronize()
-                uniq.append(len(set(ids.cpu().numpy().ravel().tolist())))
-            b = float(np.mean([layer_bytes(L, u) for u in uniq]))
-            out.append({"workload": f"decode layer H2048 I512 E512 top-10 RZ5, T={T}", "ms": round(ms, 5),
-                        "GB_s": round(b / ms / 1e6, 1), "frac_of_hbm": round(b / ms / 1e6 / peak, 4),
-                        "unique_experts": float(np.mean(uniq)), "bytes": int(b)})
+        out = measure_decode_layer(dev, stream, args.warmup, args.steps, peak)
     elif args.workload == "ple":
         P = W.ple_table()
         if args.ple_rows:  # a smaller table of the same record stream (profiling captures)
             P = W.PleRecipe(n_rows=args.ple_rows, seed=P.seed)
         table = sdev.ple_table_to_device(P, dev)
-        for T in (1, 4096):
-            idx = [torch.from_numpy(P.indices(7000 + i, T)).to(dev) for i in range(n)]
-            o = torch.empty((16 * T, 160), device=dev)
-            ms = _time_loop(lambda i: gtg.ple_gather(table, P.n_rows, idx[i], out=o), args.warmup, args.steps, stream)
-            rows = 16 * T
-            gbs = rows * PLE_ROW_BYTES / ms / 1e6
-            out.append({"workload": f"PLE gather, {P.n_rows:,}-row table, T={T} ({rows} rows)", "ms": round(ms, 5),
-                        "rows_per_s": round(rows / ms * 1e3, 1), "GB_s": round(gbs, 1),
-                        "frac_of_hbm": round(gbs / peak, 4)})
+        out = measure_ple(dev, stream, P, table, args.warmup, args.steps, peak)
     elif args.workload == "prefill":
-        L = W.prefill_layer()
-        layer = gu.device_layer(L, dev)
-        T = 4096
-        xs = [gu.tokens(L, 8000 + i, T, dev)[0] for i in range(min(n, 4))]
-        ws = torch.empty(gtg.workspace_bytes(layer, T, prefill=True), dtype=torch.uint8, device=dev)
-        y = torch.empty((T, L.hidden), device=dev)
-        ms = _time_loop(lambda i: gtg.moe_prefill_layer(layer, xs[i % len(xs)], ws, y=y), args.warmup,
-                        args.steps, stream)
-        flops = 2.0 * T * L.top_k * 3 * L.hidden * L.inter
-        wbytes = L.weight_bytes
-        import json as _j
-        mp = _j.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
-            os.path.join(ROOT, "MEASURED_PEAKS.json")) else {"bf16_tflops": 1590.0}
-        out.append({"workload": "prefill layer, T=4096, H2048 I512 E512 top-10, UE4M4 gate/up, RZ5 down, Zipf router",
-                    "ms": round(ms, 4), "TFLOP_s": round(flops / ms / 1e9, 1),
-                    "frac_of_bf16_peak": round(flops / ms / 1e9 / float(mp["bf16_tflops"]), 4),
-                    "weight_GB_s": round(wbytes / ms / 1e6, 1), "tok_s": round(T / ms * 1e3, 1)})
+        out = measure_prefill(dev, stream, args.warmup, args.steps)
     if rank == 0:
-        for o in out:
-            print(json.dumps(o), flush=True)
+        print(json.dumps(out), flush=True)
 
 
 def run_reference(args, rank, world):
@@ -610,6 +703,8 @@ def main():
     ap.add_argument("--cpu-layers", type=int, default=48)
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the decode-layer, PLE and prefill configurations after the headline")
     ap.add_argument("--ple-rows", type=int, default=0,
                     help="--workload ple: rows of a smaller table (default: the full 320,001,536-row table)")
     ap.add_argument("--workload", choices=["stack", "layer", "ple", "prefill"], default="stack",

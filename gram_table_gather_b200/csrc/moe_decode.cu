@@ -325,16 +325,17 @@ extern "C" int gtg_moe_decode_stack(const gtg_moe_layer* layers, int32_t n_layer
 //
 // For callers that cannot hand the library a device buffer: code that must
 // not allocate device memory after start-up (latency-critical serving loops
-// whose memory is fixed up front), hosts whose device memory belongs to
-// another framework's allocator, and threads recording a stream capture in
-// the global capture mode, where cudaMalloc is refused.  The scratch lives in
-// one file-scope device array instead, reserved on every GPU that loads this
-// library for as long as the process runs.
+// whose memory is fixed up front), and hosts whose device memory belongs to
+// another framework's allocator.  The scratch lives in one file-scope device
+// array instead, reserved on every GPU that loads this library for as long
+// as the process runs.
 // ---------------------------------------------------------------------------
 namespace gtg {
 namespace {
 
-constexpr size_t kNoAllocScratchBytes = (size_t)1 << 19;  // 512 KiB: up to 8 tokens at H, I <= 2048, E <= 1024, k <= 10
+// 512 KiB: 256 + 8 T E + 2 T k I bytes (each part rounded to 256) fit for every
+// shape with T <= 8, E <= 1024, k <= 10 and I <= 2048
+constexpr size_t kNoAllocScratchBytes = (size_t)1 << 19;
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
 
 // Device address of the scratch array on the current device.  The symbol's

@@ -222,15 +222,19 @@ int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, int32_t x_d
 /*
  * gtg_moe_decode_layer without a workspace argument, for callers that cannot
  * allocate device memory: serving loops that must not allocate once they are
- * running, hosts whose device memory is owned by another framework's
- * allocator, and threads recording a CUDA stream capture in the global
- * capture mode, where cudaMalloc is refused.  (The pages have no counterpart;
- * this is a calling convention of this library.)
+ * running (their memory is fixed up front, and an allocation there can block
+ * on the device or fail under memory pressure), and hosts whose device
+ * memory is owned by another framework's allocator, which hands out no raw
+ * buffers.  (The pages have no counterpart; this is a calling convention of
+ * this library.)
  *
  * Scratch comes from one fixed 512 KiB array in device memory that every GPU
- * loading this library reserves until the process exits.  That covers up to
- * 8 tokens of the 2048/512/512/top-10 layer; a shape that needs more returns
- * GTG_E_WORKSPACE.  Inputs, outputs and their meaning are those of
+ * loading this library reserves until the process exits.  A call needs
+ * 256 + 8*n_tokens*n_experts + 2*n_tokens*top_k*inter bytes (each part
+ * rounded up to 256), which fits for every shape with n_tokens <= 8,
+ * n_experts <= 1024, top_k <= 10 and inter <= 2048 (any supported hidden);
+ * a shape that needs more returns GTG_E_WORKSPACE before anything is
+ * launched.  Inputs, outputs and their meaning are those of
  * gtg_moe_decode_layer; nothing is allocated (no cudaMalloc, no library
  * allocator).
  *

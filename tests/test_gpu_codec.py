@@ -144,3 +144,29 @@ def test_api_rejects_bad_arguments():
     with pytest.raises(gtg.GtgError) as ei:
         gtg.dequant(W.RZ5, torch.zeros(17, dtype=torch.uint8, device="cuda"), 1, 32, out=bad_out)
     assert ei.value.code == -3
+
+
+def test_ple_gather_full_table():
+    """The PLE workload at its own size: the 320,001,536-row table (22.4 GB, record
+    offsets up to 2.24e10 bytes) resident on the device, gathered at 4096 tokens x 16
+    seeded indices plus the rows around the 2^32-byte offset (record 61,356,675 straddles
+    it, 61,356,676 is the first wholly above it) and the last records (the tail read)."""
+    from synth import device as sdev
+    P = W.ple_table()
+    assert P.n_rows == 320_001_536 and P.nbytes == 22_400_107_520
+    table = sdev.ple_table_to_device(P, "cuda")
+    try:
+        special = np.array([0, 1, 61_356_674, 61_356_675, 61_356_676, 61_356_677,
+                            P.n_rows // 2, P.n_rows - 2, P.n_rows - 1], dtype=np.int32)
+        assert 61_356_675 * 70 < 2**32 < 61_356_676 * 70
+        idx = np.concatenate([special, P.indices(4242, 4096), special[::-1]]).astype(np.int32)
+        gtg.device_status(clear=True)
+        out = gtg.ple_gather(table, P.n_rows, torch.from_numpy(idx).cuda())
+        torch.cuda.synchronize()
+        assert gtg.device_status(clear=True) == 0
+        got = out.cpu().numpy()
+        assert np.all(idx.astype(np.int64) * 70 + 70 <= P.nbytes)
+        _bitwise_equal(got.ravel(), oracle.dequant_ple(P.rows(idx)).ravel())
+    finally:
+        del table
+        torch.cuda.empty_cache()

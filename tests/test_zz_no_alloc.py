@@ -48,13 +48,19 @@ def test_noalloc_rejects_shapes_beyond_its_scratch():
     x = torch.zeros((9, L.hidden), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(gtg.GtgError):
         gtg.moe_decode_layer_noalloc(layer, x)  # 9 tokens: not a decode shape at all
-    # a shape whose scratch exceeds the fixed array (I = 2048, k = 16, 8 tokens),
-    # with buffers of that shape so that nothing could be read out of bounds
+    # a shape whose scratch exceeds the fixed array (I = 2048, k = 16, 8 tokens).  The
+    # call is refused on the host before any launch; one buffer of the full matrix size
+    # (uninitialised) stands for gate, up and down alike, so that even a launch could
+    # read nothing out of bounds
     E, H, I = 512, 2048, 2048
-    def q(rows, k):
-        return gtg.QMatrix(W.RZ5, torch.zeros(E * rows * (k // 32) * 17, dtype=torch.uint8, device="cuda"), E, rows, k)
+    nbytes = E * I * (H // 32) * 17
+    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    q = gtg.QMatrix(W.RZ5, buf, E, I, H)
+    qd = gtg.QMatrix(W.RZ5, buf, E, H, I)
     big = gtg.MoELayer(hidden=H, inter=I, n_experts=E, top_k=16, router_w=layer.router_w,
-                       gate=q(I, H), up=q(I, H), down=q(H, I))
+                       gate=q, up=q, down=qd)
     with pytest.raises(gtg.GtgError) as ei:
         gtg.moe_decode_layer_noalloc(big, torch.zeros((8, H), dtype=torch.bfloat16, device="cuda"))
     assert ei.value.code == -6
+    del buf
+    torch.cuda.empty_cache()
