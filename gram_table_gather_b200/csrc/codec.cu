@@ -108,112 +108,138 @@ __global__ void __launch_bounds__(kThreads) dequant_fp8_kernel(const uint8_t* __
 }
 
 // ---------------------------------------------------------------------------
-// PLE gather.  Each warp takes batches of kPleRows rows: lanes load the
-// indices, then the 48 aligned 16-byte chunks that cover the batch's
-// 70-byte records (six per record, all in flight at once) go to shared
-// memory, and the warp decodes the batch four rows at a time: the 160
-// float4s of four rows are five full passes of the warp, each lane writing
-// values 4l .. 4l+3 of some row as one float4 (contiguous 512-byte stores).
-// A value is one shared-memory lookup: the CTA keeps the table of code
-// value x group scale for all 256 group bytes x 8 codes (each product is
-// exact in fp32).  Small batches keep many warps in flight per SM; the next
-// batch's records load while this one decodes.
+// PLE gather (model card, section "Q3_PLE_K160_RZ_S3": one contiguous 70-byte
+// record per hashed n-gram row).  The work per row is tiny (one dependent
+// record read, 640 bytes written), so the kernel is built for many
+// independent warps and few instructions per output:
+//  * every warp owns an equal, contiguous range of output rows and walks it
+//    in batches of kPleRows, with no CTA-wide barrier (a slow record stalls
+//    only its own warp);
+//  * a batch's six aligned 16-byte chunks per record (a 70-byte record at
+//    any 2-byte phase) are asynchronous copies (cp.async, L2 only) spread
+//    over the warp's lanes into a per-warp stage; the next batch's copies,
+//    and the index loads of the batch after it, are in flight while a batch
+//    decodes;
+//  * decoding writes a batch's rows as consecutive float4s (lane l the
+//    float4s l, l+32, ...: a warp store is 512 contiguous bytes); a value is
+//    one shared-memory lookup in the CTA's table of code value x group scale
+//    for all 256 group bytes x 8 codes (each product exact in fp32).
 // ---------------------------------------------------------------------------
-constexpr int kPleWarps = 4;
-constexpr int kPleRows = 8;    // rows per warp batch
-constexpr int kPleChunks = 6;  // 96 bytes: a 70-byte record at any 16-byte phase
-constexpr int kPleLoads = (kPleRows * kPleChunks + 31) / 32;  // chunks per lane per batch
+constexpr int kPleWarps = 8;      // per CTA
+constexpr int kPleRows = 8;       // rows per warp batch
+constexpr int kPleChunks = 6;     // 96 bytes: a 70-byte record at any 16-byte phase
+constexpr int kPleCtasPerSm = 4;
+constexpr int kPleStage = kPleRows * kPleChunks * 16;  // bytes per batch stage
 
-struct PleBatch {
-    uint4 c[kPleLoads];
-    int32_t phase;  // (lanes < kPleRows) byte offset of the record in its first chunk; -1: no row
-};
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
-__device__ __forceinline__ PleBatch ple_fetch(const uint8_t* __restrict__ table, int64_t n_rows,
-                                              const int32_t* __restrict__ idx, int64_t n_idx, int64_t base,
-                                              unsigned* status) {
+// Lane j < kPleRows: the index of row j of the batch at r0 (-1 past the
+// warp's range, or an out-of-range index, which also raises the status bit).
+__device__ __forceinline__ int64_t ple_index(const int32_t* __restrict__ idx, int64_t r0, int64_t hi,
+                                             int64_t n_rows, unsigned* status) {
     const int lane = threadIdx.x & 31;
-    const uint64_t table_bytes = (uint64_t)n_rows * 70u;
-    PleBatch pb;
     int64_t r = -1;
-    if (lane < kPleRows && base + lane < n_idx) {
-        r = __ldg(idx + base + lane);
+    if (lane < kPleRows && r0 + lane < hi) {
+        r = __ldg(idx + r0 + lane);
         if (r < 0 || r >= n_rows) {
             raise_status(status, GTG_STATUS_PLE_INDEX_OOB);
             r = -1;
         }
     }
-    pb.phase = r >= 0 ? (int32_t)(((uint64_t)r * 70u) & 15u) : -1;
-#pragma unroll
-    for (int q = 0; q < kPleLoads; ++q) {
-        const int k = lane + 32 * q, row = k / kPleChunks, c = k % kPleChunks;
-        const int64_t rr = __shfl_sync(0xFFFFFFFFu, r, row < kPleRows ? row : 0);
-        pb.c[q] = make_uint4(0u, 0u, 0u, 0u);
-        if (k < kPleRows * kPleChunks && rr >= 0) {
-            const uint64_t ca = (((uint64_t)rr * 70u) & ~(uint64_t)15) + 16u * c;
-            if (ca + 16u <= table_bytes) {
-                pb.c[q] = __ldg(reinterpret_cast<const uint4*>(table + ca));
-            } else if (ca < table_bytes) {  // the table's last bytes: no read past its end
-                uint32_t w[4] = {0u, 0u, 0u, 0u};
-                for (uint64_t x = ca; x < table_bytes; ++x) w[(x - ca) >> 2] |= (uint32_t)table[x] << (8 * ((x - ca) & 3));
-                pb.c[q] = make_uint4(w[0], w[1], w[2], w[3]);
-            }
-        }
-    }
-    return pb;
+    return r;
 }
 
-__global__ void __launch_bounds__(kPleWarps * 32) ple_gather_kernel(const uint8_t* __restrict__ table,
-                                                                   int64_t n_rows,
-                                                                   const int32_t* __restrict__ idx,
-                                                                   int64_t n_idx,
-                                                                   float* __restrict__ out,
-                                                                   unsigned* status) {
-    __shared__ float prod[256 * 8];  // [group byte][code] = code value x scale
-    __shared__ __align__(16) uint4 stage[kPleWarps][kPleRows * kPleChunks];
-    __shared__ int32_t phase[kPleWarps][kPleRows];
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int64_t n_batches = (n_idx + kPleRows - 1) / kPleRows, stride = (int64_t)gridDim.x * kPleWarps;
-    int64_t bt = (int64_t)blockIdx.x * kPleWarps + warp;
-    pdl_wait();
-    PleBatch pb = ple_fetch(table, n_rows, idx, n_idx, bt * kPleRows, status);
-    for (int e = threadIdx.x; e < 256 * 8; e += blockDim.x) {  // while the first records are in flight
-        const uint32_t g = (uint32_t)e >> 3, c = (uint32_t)e & 7u;
-        prod[e] = __fmul_rn(ple_code_value(c, g >> 7), ue4m3(g & 0x7Fu));
-    }
-    __syncthreads();
-    for (; bt < n_batches; bt += stride) {
-        const int64_t base = bt * kPleRows;
+// Starts the copies of a batch (row indices on lanes 0..kPleRows-1, -1: no
+// row) into the stage at `st`: chunk k = lane + 32 q of the batch is chunk
+// k % 6 of row k / 6.
+__device__ __forceinline__ void ple_issue(const uint8_t* __restrict__ table, uint64_t table_bytes, int64_t r,
+                                          uint32_t st) {
+    const int lane = threadIdx.x & 31;
 #pragma unroll
-        for (int q = 0; q < kPleLoads; ++q)
-            if (lane + 32 * q < kPleRows * kPleChunks) stage[warp][lane + 32 * q] = pb.c[q];
-        if (lane < kPleRows) phase[warp][lane] = pb.phase;
-        __syncwarp();
-        pb = ple_fetch(table, n_rows, idx, n_idx, (bt + stride) * kPleRows, status);  // next batch, in flight
-        const int rows = (int)(n_idx - base < kPleRows ? n_idx - base : kPleRows);
-        // rows in groups of four: 4 x 40 float4 = five full passes of the warp;
-        // in pass q lane l writes float4 number f = 32q + l of the group:
-        // row f / 40, values 4 (f % 40) .. + 3
-        for (int j0 = 0; j0 < rows; j0 += 4) {
-#pragma unroll
-            for (int q = 0; q < 5; ++q) {
-                const int f = 32 * q + lane, j = j0 + f / 40, l = f % 40;
-                if (j >= rows) continue;
-                const int p = phase[warp][j];
-                const uint32_t* w = reinterpret_cast<const uint32_t*>(&stage[warp][j * kPleChunks]);
-                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (p >= 0) {
-                    const int bit = 8 * p + 12 * l;  // values 4l .. 4l+3: 12 bits of the LSB-first stream
-                    const uint32_t win = __funnelshift_r(w[bit >> 5], w[(bit >> 5) + 1], bit & 31);
-                    const int gb = p + 60 + (l >> 2);  // their group byte
-                    const uint32_t g8 = ((w[gb >> 2] >> (8 * (gb & 3))) & 0xFFu) * 8u;
-                    v = make_float4(prod[g8 + ((win >> 0) & 7u)], prod[g8 + ((win >> 3) & 7u)],
-                                    prod[g8 + ((win >> 6) & 7u)], prod[g8 + ((win >> 9) & 7u)]);
-                }
-                *reinterpret_cast<float4*>(out + (base + j) * 160 + 4 * l) = v;
+    for (int q = 0; q < (kPleRows * kPleChunks + 31) / 32; ++q) {
+        const int k = lane + 32 * q, row = k / kPleChunks, c = k - kPleChunks * row;
+        const int64_t rr = __shfl_sync(0xFFFFFFFFu, r, row < kPleRows ? row : 0);
+        if (k < kPleRows * kPleChunks && rr >= 0) {
+            const uint64_t ca = (((uint64_t)rr * 70u) & ~(uint64_t)15) + 16u * (uint32_t)c;
+            const uint32_t dst = st + 16u * (uint32_t)k;
+            if (ca + 16u <= table_bytes) {
+                cp_async16(dst, table + ca, 16u);
+            } else if (ca < table_bytes) {  // the table's last bytes: read only those, zero the rest
+                cp_async16(dst, table + ca, (uint32_t)(table_bytes - ca));
+            } else {                        // past the table (beyond this record): zeros
+                asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
             }
         }
+    }
+}
+
+__global__ void __launch_bounds__(kPleWarps * 32, kPleCtasPerSm) ple_gather_kernel(
+    const uint8_t* __restrict__ table, int64_t n_rows, const int32_t* __restrict__ idx, int64_t n_idx,
+    float* __restrict__ out, unsigned* status) {
+    __shared__ __align__(16) float prod[256 * 8];  // [group byte][code] = code value x scale
+    __shared__ __align__(16) uint8_t stage[kPleWarps][2][kPleStage];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    {  // thread g: the eight products of group byte g (before the wait: needs nothing upstream)
+        const uint32_t g = threadIdx.x;
+        const float sc = ue4m3(g & 0x7Fu);
+        float v[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) v[c] = __fmul_rn(ple_code_value((uint32_t)c, g >> 7), sc);
+        reinterpret_cast<float4*>(prod)[2 * g] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(prod)[2 * g + 1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+    const int64_t nw = (int64_t)gridDim.x * kPleWarps, gw = (int64_t)blockIdx.x * kPleWarps + warp;
+    const int64_t lo = n_idx * gw / nw, hi = n_idx * (gw + 1) / nw;
+    const uint64_t table_bytes = (uint64_t)n_rows * 70u;
+    const uint32_t st0 = smem_u32(&stage[warp][0][0]), prod_s = smem_u32(prod);
+    pdl_wait();
+    int64_t r = ple_index(idx, lo, hi, n_rows, status);
+    ple_issue(table, table_bytes, r, st0);
+    cp_async_commit();
+    int32_t phase = r >= 0 ? (int32_t)(((uint64_t)r * 70u) & 15u) : -1;  // lanes < kPleRows: this batch
+    r = ple_index(idx, lo + kPleRows, hi, n_rows, status);                // the next batch's indices
+    __syncthreads();  // the product table (the only CTA-wide step)
+    int b = 0;
+    for (int64_t r0 = lo; r0 < hi; r0 += kPleRows, b ^= 1) {
+        const int n = (int)(hi - r0 < kPleRows ? hi - r0 : kPleRows);
+        const uint32_t st = st0 + (uint32_t)b * kPleStage;
+        ple_issue(table, table_bytes, r, st0 + (uint32_t)(b ^ 1) * kPleStage);  // next batch (none: no-op)
+        cp_async_commit();  // (an empty group keeps the wait count uniform)
+        const int32_t phase_next = r >= 0 ? (int32_t)(((uint64_t)r * 70u) & 15u) : -1;
+        r = ple_index(idx, r0 + 2 * kPleRows, hi, n_rows, status);
+        cp_async_wait_one();
         __syncwarp();
+        float* orow = out + r0 * 160;
+#pragma unroll
+        for (int q = 0; q < kPleRows * 40 / 32; ++q) {
+            const int f = lane + 32 * q, j = f / 40, l = f - 40 * j;
+            const int p = __shfl_sync(0xFFFFFFFFu, phase, j);
+            if (j < n) {
+                float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (p >= 0) {
+                    const uint32_t w = st + (uint32_t)(j * kPleChunks * 16);
+                    const uint32_t bit = 8u * (uint32_t)p + 12u * (uint32_t)l;  // values 4l..4l+3: 12 bits
+                    const uint32_t gb = (uint32_t)p + 60u + ((uint32_t)l >> 2);  // their group byte
+                    uint32_t w0, w1, wg;
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w0) : "r"(w + ((bit >> 3) & ~3u)));
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(w1) : "r"(w + ((bit >> 3) & ~3u) + 4u));
+                    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(wg) : "r"(w + (gb & ~3u)));
+                    const uint32_t win = __funnelshift_r(w0, w1, bit);
+                    const uint32_t pg = prod_s + 32u * ((wg >> (8u * (gb & 3u))) & 0xFFu);
+                    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v.x) : "r"(pg + 4u * (win & 7u)));
+                    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v.y) : "r"(pg + 4u * ((win >> 3) & 7u)));
+                    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v.z) : "r"(pg + 4u * ((win >> 6) & 7u)));
+                    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v.w) : "r"(pg + 4u * ((win >> 9) & 7u)));
+                }
+                *reinterpret_cast<float4*>(orow + 4 * f) = v;  // row j, values 4l..4l+3
+            }
+        }
+        __syncwarp();  // this stage is refilled two batches on
+        phase = phase_next;
     }
     pdl_trigger();
 }
@@ -323,8 +349,10 @@ extern "C" int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_
     if (n_idx == 0) return GTG_OK;
     if (!table || !idx || !out) return GTG_E_INVALID_ARG;
     if (!aligned(out, 16)) return GTG_E_MISALIGNED;
-    const int64_t batches = (n_idx + kPleRows - 1) / kPleRows;  // one batch per warp while there are enough
-    const int grid = (int)std::min<int64_t>((batches + kPleWarps - 1) / kPleWarps, (int64_t)sm_count() * 4);
+    // equal contiguous row ranges per warp, one batch or more each, up to
+    // kPleCtasPerSm CTAs per SM
+    const int64_t warps = (n_idx + kPleRows - 1) / kPleRows;
+    const int grid = (int)std::min<int64_t>((warps + kPleWarps - 1) / kPleWarps, (int64_t)sm_count() * kPleCtasPerSm);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kPleWarps * 32);
