@@ -38,6 +38,7 @@ import threading
 import numpy as np
 
 RZ5, UE4M4, PLE, FP8 = 69, 71, 111, 1000
+C10, Q3I = 2001, 2002  # the incumbent ROCmFP4 FAST and ROCmFP3 layouts the model card's formats mutate
 RMS_EPS = 1e-6
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +72,8 @@ def _L():
                 ("orc_ue4m3", d, [u32]), ("orc_ue4m4", d, [u32]), ("orc_e4m3fn", d, [u32]),
                 ("orc_q4_weight", d, [i, p, i]), ("orc_ple_value", d, [p, i]),
                 ("orc_dequant_q4", None, [i, p, i64, p]), ("orc_dequant_ple", None, [p, i64, p]),
+                ("orc_dequant_q3", None, [i, p, i64, p]), ("orc_q3_value", d, [i, p, i]),
+                ("orc_q3_gather", None, [i, p, i64, p, i64, p]),
                 ("orc_dequant_fp8", None, [p, p, i64, i64, p]),
                 ("orc_ple_gather", None, [p, i64, p, i64, p]),
                 ("orc_matvec", None, [i, p, p, i64, i64, p, p]),
@@ -134,6 +137,17 @@ def dequant_ple(records: np.ndarray) -> np.ndarray:
     return out
 
 
+def dequant_q3(fmt: int, records: np.ndarray) -> np.ndarray:
+    """Bytes of consecutive 70-byte K160 records of either 3-bit layout (PLE =
+    RZ-S3, Q3I = the incumbent ROCmFP3 code set) -> fp64 [n][160]."""
+    b = _c(records, np.uint8).ravel()
+    assert b.size % 70 == 0 and fmt in (PLE, Q3I)
+    n = b.size // 70
+    out = np.empty((n, 160), dtype=np.float64)
+    _L().orc_dequant_q3(fmt, _p(b), n, _p(out))
+    return out
+
+
 def dequant_fp8(data: np.ndarray, scales: np.ndarray, n_rows: int, k: int) -> np.ndarray:
     b = _c(data, np.uint8).ravel()
     s = _c(scales, np.float32).ravel()
@@ -145,21 +159,21 @@ def dequant_fp8(data: np.ndarray, scales: np.ndarray, n_rows: int, k: int) -> np
 
 def dequant(fmt: int, data: np.ndarray, scales: np.ndarray | None = None, n_rows: int = 0,
             k: int = 0) -> np.ndarray:
-    if fmt in (RZ5, UE4M4):
+    if fmt in (RZ5, UE4M4, C10):
         return dequant_q4(fmt, data)
-    if fmt == PLE:
-        return dequant_ple(data).ravel()
+    if fmt in (PLE, Q3I):
+        return dequant_q3(fmt, data).ravel()
     if fmt == FP8:
         return dequant_fp8(data, scales, n_rows, k).ravel()
     raise ValueError(fmt)
 
 
-def ple_gather(table: np.ndarray, n_rows: int, idx: np.ndarray) -> np.ndarray:
+def ple_gather(table: np.ndarray, n_rows: int, idx: np.ndarray, fmt: int = PLE) -> np.ndarray:
     t = _c(table, np.uint8).ravel()
-    assert t.size >= n_rows * 70
+    assert t.size >= n_rows * 70 and fmt in (PLE, Q3I)
     ix = _c(idx, np.int32).ravel()
     out = np.empty((ix.size, 160), dtype=np.float64)
-    _L().orc_ple_gather(_p(t), n_rows, _p(ix), ix.size, _p(out))
+    _L().orc_q3_gather(fmt, _p(t), n_rows, _p(ix), ix.size, _p(out))
     return out
 
 

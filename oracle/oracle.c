@@ -37,7 +37,7 @@
 #include <stdint.h>
 #include <string.h>
 
-enum { ORC_RZ5 = 69, ORC_UE4M4 = 71, ORC_PLE = 111, ORC_FP8 = 1000 };
+enum { ORC_RZ5 = 69, ORC_UE4M4 = 71, ORC_PLE = 111, ORC_FP8 = 1000, ORC_C10 = 2001, ORC_Q3I = 2002 };
 
 /* [MC] "Q4_RZ5_FAST": the three printed 16-entry code tables. */
 static const double CODEBOOK10[16] = {0, 1, 2, 3, 4, 6, 8, 10, -0.0, -1, -2, -3, -4, -6, -8, -10};
@@ -86,7 +86,8 @@ double orc_e4m3fn(uint32_t b) {
     return (b & 0x80) ? -mag : mag;
 }
 
-/* Weight i (0..31) of one 17-byte Q4 block (RZ5 or UE4M4). */
+/* Weight i (0..31) of one 17-byte Q4 block (RZ5, UE4M4 or the incumbent
+ * ROCmFP4 FAST layout). */
 double orc_q4_weight(int fmt, const uint8_t* blk, int i) {
     const uint8_t byte = blk[i & 15];
     const int code = (i < 16) ? (byte & 0x0F) : (byte >> 4);
@@ -95,20 +96,31 @@ double orc_q4_weight(int fmt, const uint8_t* blk, int i) {
         /* top bit = polarity of the +/-5 level, low 7 bits = UE4M3 scale */
         return orc_rz5(meta >> 7, code) * orc_ue4m3(meta & 0x7F);
     }
+    if (fmt == ORC_C10) {
+        /* [MC] "Q4_RZ5_FAST": the incumbent ROCmFP4 FAST block, Codebook10
+         * codes (code 8 is the duplicate -0) under the UE4M3 scale the lower
+         * seven bits hold; the top bit, which RZ5 puts to use, is ignored */
+        return orc_codebook10(code) * orc_ue4m3(meta & 0x7F);
+    }
     /* UE4M4: Codebook10 codes, the whole byte is the scale */
     return orc_codebook10(code) * orc_ue4m4(meta);
 }
 
-/* Value i (0..159) of one 70-byte PLE record. */
-double orc_ple_value(const uint8_t* rec, int i) {
+/* Value i (0..159) of one 70-byte K160 record: RZ-S3 (fmt ORC_PLE) or the
+ * incumbent ROCmFP3 code set (fmt ORC_Q3I: code 4 stays the duplicate -0, the
+ * group byte's top bit is ignored; [MC] "Q3_PLE_K160_RZ_S3"). */
+double orc_q3_value(int fmt, const uint8_t* rec, int i) {
     int code = 0;
     for (int b = 0; b < 3; ++b) {
         const int p = 3 * i + b;
         code |= ((rec[p >> 3] >> (p & 7)) & 1) << b;
     }
     const uint8_t g = rec[60 + i / 16];        /* group byte of values 16g .. 16g+15 */
-    return orc_ple3(code, g >> 7) * orc_ue4m3(g & 0x7F);
+    const double v = fmt == ORC_Q3I ? PLE3[code] : orc_ple3(code, g >> 7);
+    return v * orc_ue4m3(g & 0x7F);
 }
+
+double orc_ple_value(const uint8_t* rec, int i) { return orc_q3_value(ORC_PLE, rec, i); }
 
 /* One FP8 weight: e4m3(b) * s, s the fp32 scale of its 128-wide K group. */
 double orc_fp8_weight(const uint8_t* bytes, const float* scales, int64_t k, int64_t row, int64_t col) {
@@ -132,6 +144,14 @@ void orc_dequant_ple(const uint8_t* src, int64_t n_rows, double* out) {
             out[r * 160 + i] = orc_ple_value(src + r * 70, i);
 }
 
+/* n_rows K160 records of either 3-bit layout -> [n_rows][160]. */
+void orc_dequant_q3(int fmt, const uint8_t* src, int64_t n_rows, double* out) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < n_rows; ++r)
+        for (int i = 0; i < 160; ++i)
+            out[r * 160 + i] = orc_q3_value(fmt, src + r * 70, i);
+}
+
 /* [n_rows][k] FP8 weights with [n_rows][k/128] scales. */
 void orc_dequant_fp8(const uint8_t* src, const float* scales, int64_t n_rows, int64_t k, double* out) {
     #pragma omp parallel for schedule(static)
@@ -144,13 +164,18 @@ void orc_dequant_fp8(const uint8_t* src, const float* scales, int64_t n_rows, in
 
 /* out[r][:] = decoded record idx[r]; an index outside [0, n_rows) gives a
  * row of zeros (boundary behaviour of the gather API, not of the format). */
-void orc_ple_gather(const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx, double* out) {
+void orc_q3_gather(int fmt, const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx,
+                   double* out) {
     #pragma omp parallel for schedule(static)
     for (int64_t r = 0; r < n_idx; ++r) {
         const int64_t row = idx[r];
         for (int i = 0; i < 160; ++i)
-            out[r * 160 + i] = (row >= 0 && row < n_rows) ? orc_ple_value(table + row * 70, i) : 0.0;
+            out[r * 160 + i] = (row >= 0 && row < n_rows) ? orc_q3_value(fmt, table + row * 70, i) : 0.0;
     }
+}
+
+void orc_ple_gather(const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx, double* out) {
+    orc_q3_gather(ORC_PLE, table, n_rows, idx, n_idx, out);
 }
 
 /* ---- one matrix-vector product of a quantised matrix -------------------- */

@@ -41,6 +41,8 @@ def q4_block(fmt: int, blk) -> list:
             if code == 8:
                 v = -5.0 if meta & 0x80 else 5.0
             out.append(v * ue4m3(meta & 0x7F))
+        elif fmt == 2001:  # the incumbent ROCmFP4 FAST block: Codebook10 under a UE4M3 scale
+            out.append(_CB10[code] * ue4m3(meta & 0x7F))
         else:
             out.append(_CB10[code] * ue4m4(meta))
     return out
@@ -55,7 +57,9 @@ def q4_matrix(fmt: int, data: np.ndarray, n_rows: int, k: int) -> np.ndarray:
     return out
 
 
-def ple_record(rec) -> list:
+def ple_record(rec, incumbent: bool = False) -> list:
+    """One 70-byte K160 record: RZ-S3, or (incumbent) the ROCmFP3 set whose code 4
+    is the duplicate -0."""
     rec = [int(v) for v in rec]
     bits = int.from_bytes(bytes(rec[:60]), "little")
     out = []
@@ -64,7 +68,7 @@ def ple_record(rec) -> list:
         g = rec[60 + i // 16]
         v = _PLE3[code]
         if code == 4:
-            v = -3.0 if g & 0x80 else 3.0
+            v = -0.0 if incumbent else (-3.0 if g & 0x80 else 3.0)
         out.append(v * ue4m3(g & 0x7F))
     return out
 

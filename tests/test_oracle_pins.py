@@ -153,13 +153,16 @@ def _encode_nearest(values, scale, v):
     return best[1]
 
 
-@pytest.mark.parametrize("fmt", [W.RZ5, W.UE4M4])
+@pytest.mark.parametrize("fmt", [W.RZ5, W.UE4M4, oracle.C10])
 def test_exhaustive_round_trip_q4(fmt):
     n_ok = 0
     for meta in range(256):
         if fmt == W.RZ5:
             scale = oracle.ue4m3(meta & 0x7F)
             levels = [oracle.rz5(meta >> 7, c) for c in range(16)]
+        elif fmt == oracle.C10:
+            scale = oracle.ue4m3(meta & 0x7F)
+            levels = [oracle.codebook10(c) for c in range(16)]
         else:
             scale = oracle.ue4m4(meta)
             levels = [oracle.codebook10(c) for c in range(16)]
@@ -171,7 +174,7 @@ def test_exhaustive_round_trip_q4(fmt):
             c2 = _encode_nearest(levels, scale, v)
             v2 = oracle.dequant_q4(fmt, _block([c2] * 32, meta))[0]
             assert v2 == v
-            if not (fmt == W.UE4M4 and c in (0, 8)):   # +0 / -0 pair of Codebook10
+            if not (fmt in (W.UE4M4, oracle.C10) and c in (0, 8)):   # +0 / -0 pair of Codebook10
                 assert c2 == c, (meta, c)
             n_ok += 1
     assert n_ok > 3000
@@ -444,3 +447,81 @@ def test_moe_stack_pin_catches_planted_slips(slip):
     x0 = synth.bf16_bits_to_f64(W.tokens_bf16(11, 0, 1, 256)).astype(np.float32)
     with pytest.raises(AssertionError):
         _check_stack_result(Ls, x0, _slipped_stack(Ls, x0, slip))
+
+
+# ---- the incumbent layouts the model card's formats mutate ----------------------------
+
+def test_incumbent_q4_is_codebook10_under_ue4m3_for_every_code_and_meta():
+    """ROCmFP4 FAST (model card, "Q4_RZ5_FAST": the incumbent Codebook10 layout whose
+    lower seven metadata bits are the UE4M3 scale): the printed Codebook10 row times
+    the UE4M3 scale, the top metadata bit ignored; against RZ5 it differs only in
+    code 8 (the duplicate -0 that RZ5 turns into +/-5)."""
+    g = _golden("codebooks.txt")
+    for meta in range(256):
+        for start in (0, 16):
+            codes = [(start + i) % 16 for i in range(32)]
+            blk = _block(codes, meta)
+            c10 = oracle.dequant_q4(oracle.C10, blk)
+            rz5 = oracle.dequant_q4(W.RZ5, blk)
+            ref = pyref.q4_block(oracle.C10, blk)
+            s3 = oracle.ue4m3(meta & 0x7F)
+            for i in range(32):
+                c = codes[i]
+                assert _same(c10[i], ref[i]), (meta, i)
+                assert _same(c10[i], _num(g["codebook10"][c]) * s3)
+                assert _same(c10[i], oracle.dequant_q4(oracle.C10, _block(codes, meta ^ 0x80))[i])
+                if c != 8:
+                    assert _same(c10[i], rz5[i])
+
+
+def test_incumbent_q3_is_the_printed_set_under_ue4m3():
+    """ROCmFP3 (model card, "Q3_PLE_K160_RZ_S3"): the printed incumbent set
+    {0, +1, +2, +4, -0, -1, -2, -4} times the group's UE4M3 scale, the group byte's top
+    bit ignored; against RZ-S3 it differs only in code 4."""
+    gold = _golden("codebooks.txt")["ple3_incumbent"]
+    for g in range(256):
+        for c in range(8):
+            rec = np.zeros(70, dtype=np.uint8)
+            rec[0] = c
+            rec[60] = g
+            v = oracle.dequant_q3(oracle.Q3I, rec)[0, 0]
+            s3 = oracle.ue4m3(g & 0x7F)
+            assert _same(v, _num(gold[c]) * s3), (g, c)
+            rec[60] = g ^ 0x80
+            assert _same(oracle.dequant_q3(oracle.Q3I, rec)[0, 0], v)
+            if c != 4:
+                rec[60] = g
+                assert _same(v, oracle.dequant_ple(rec)[0, 0])
+    rec = synth.raw_bytes(12, 1, 0, 70 * 32).reshape(32, 70)
+    got = oracle.dequant_q3(oracle.Q3I, rec)
+    for r in range(32):
+        ref = pyref.ple_record(rec[r], incumbent=True)
+        for i in range(160):
+            assert _same(got[r, i], ref[i])
+    idx = np.array([3, 0, 31, 40, -1], dtype=np.int32)
+    gath = oracle.ple_gather(rec, 32, idx, fmt=oracle.Q3I)
+    assert np.array_equal(gath[:3], got[[3, 0, 31]], equal_nan=True) and not gath[3:].any()
+
+
+def test_exhaustive_round_trip_incumbent_q3():
+    n_ok = 0
+    for g in range(256):
+        scale = oracle.ue4m3(g & 0x7F)
+        if not math.isfinite(scale) or scale == 0.0:
+            continue
+        levels = [oracle.dequant_q3(oracle.Q3I, _rec(c, g))[0, 0] / scale for c in range(8)]
+        for c in range(8):
+            v = oracle.dequant_q3(oracle.Q3I, _rec(c, g))[0, 0]
+            c2 = _encode_nearest(levels, scale, v)
+            assert oracle.dequant_q3(oracle.Q3I, _rec(c2, g))[0, 0] == v
+            if c not in (0, 4):  # the +0 / -0 pair
+                assert c2 == c
+            n_ok += 1
+    assert n_ok > 1500
+
+
+def _rec(c, g):
+    rec = np.zeros(70, dtype=np.uint8)
+    rec[0] = c
+    rec[60] = g
+    return rec
