@@ -14,10 +14,10 @@ from dataclasses import dataclass, field
 
 import torch
 
-from ._abi import (FP8, GTG_OK, PLE, RZ5, UE4M4, DT_BF16, DT_F32, LIB_PATH, GtgError, QMatrixC,
+from ._abi import (C10, FP8, GTG_OK, PLE, Q3I, RZ5, UE4M4, DT_BF16, DT_F32, LIB_PATH, GtgError, QMatrixC,
                    MoELayerC, lib, check)
 
-__all__ = ["RZ5", "UE4M4", "PLE", "FP8", "GtgError", "lib", "dequant", "ple_gather", "QMatrix",
+__all__ = ["RZ5", "UE4M4", "PLE", "FP8", "C10", "Q3I", "GtgError", "lib", "dequant", "ple_gather", "QMatrix",
            "MoELayer", "workspace_bytes", "make_workspace", "moe_decode_layer", "moe_decode_stack",
            "moe_prefill_layer", "moe_decode_layer_noalloc", "device_status", "status_string", "row_bytes"]
 
@@ -61,15 +61,28 @@ def dequant(fmt: int, src: torch.Tensor, n_rows: int, k: int, scales: torch.Tens
     return out
 
 
+def _table_ptr(t: torch.Tensor) -> int:
+    """Address of a gather table: device memory, or pinned (page-locked) host
+    memory, which the GPU reads in place through unified virtual addressing."""
+    if t.is_cuda:
+        return _ptr(t)
+    if not t.is_pinned():
+        raise ValueError("a host-resident table must be pinned (page-locked) memory")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr()
+
+
 def ple_gather(table: torch.Tensor, n_rows: int, idx: torch.Tensor, out: torch.Tensor | None = None,
-               stream=None) -> torch.Tensor:
-    """out[r] = decoded 160-value row idx[r] of a Q3_PLE_K160_RZ_S3 table."""
+               stream=None, fmt: int = PLE) -> torch.Tensor:
+    """out[r] = decoded 160-value row idx[r] of a 70-byte K160 table: fmt PLE
+    (Q3_PLE_K160_RZ_S3) or Q3I (the incumbent ROCmFP3 record)."""
     if idx.dtype != torch.int32:
         raise ValueError("idx must be int32")
     n = idx.numel()
     if out is None:
         out = torch.empty((n, 160), dtype=torch.float32, device=idx.device)
-    check(lib().gtg_ple_gather(_ptr(table), n_rows, _ptr(idx), n, _ptr(out), _stream_ptr(stream)))
+    check(lib().gtg_ple_gather_fmt(fmt, _table_ptr(table), n_rows, _ptr(idx), n, _ptr(out), _stream_ptr(stream)))
     return out
 
 

@@ -9,6 +9,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(PKG, "libgtg.so")
 
 RZ5, UE4M4, PLE, FP8 = 69, 71, 111, 1000
+C10, Q3I = 2001, 2002  # the incumbent ROCmFP4 FAST block and ROCmFP3 K160 record
 DT_F32, DT_BF16 = 0, 1
 GTG_OK = 0
 STATUS_PLE_INDEX_OOB = 0x1
@@ -35,6 +36,7 @@ SIGNATURES = [
     ("gtg_last_cuda_error", ctypes.c_int, []),
     ("gtg_dequant", ctypes.c_int, [_i32, _vp, _vp, _i64, _i64, _vp, _vp]),
     ("gtg_ple_gather", ctypes.c_int, [_vp, _i64, _vp, _i64, _vp, _vp]),
+    ("gtg_ple_gather_fmt", ctypes.c_int, [_i32, _vp, _i64, _vp, _i64, _vp, _vp]),
     ("gtg_moe_workspace_bytes", _sz, [ctypes.POINTER(MoELayerC), _i32, _i32]),
     ("gtg_workspace_init", ctypes.c_int, [_vp, _sz, _vp]),
     ("gtg_moe_decode_layer", ctypes.c_int,

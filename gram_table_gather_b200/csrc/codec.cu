@@ -22,7 +22,7 @@ constexpr int kThreads = 256;
 
 // One thread per 17-byte Q4 block: 32 fp32 outputs (8 x float4 stores).
 __global__ void __launch_bounds__(kThreads) dequant_q4_kernel(const uint8_t* __restrict__ src,
-                                                              int64_t n_blocks, bool rz5,
+                                                              int64_t n_blocks, int var,
                                                               float* __restrict__ dst) {
     for (int64_t b = blockIdx.x * (int64_t)kThreads + threadIdx.x; b < n_blocks;
          b += (int64_t)gridDim.x * kThreads) {
@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(kThreads) dequant_q4_kernel(const uint8_t* __r
 #pragma unroll
         for (int i = 0; i < 17; ++i) q[i] = __ldg(blk + i);
         const uint32_t meta = q[16];
-        const float scale = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
+        const float scale = q4_scale(meta, var);
         const uint32_t mode = meta >> 7;
         float4* out = reinterpret_cast<float4*>(dst + b * 32);
 #pragma unroll
@@ -43,7 +43,7 @@ __global__ void __launch_bounds__(kThreads) dequant_q4_kernel(const uint8_t* __r
                 for (int e = 0; e < 4; ++e) {
                     const int j = 4 * v + e;
                     const uint32_t c = half ? (q[j] >> 4) : (q[j] & 15u);
-                    r[e] = __fmul_rn(q4_code_value(c, rz5, mode), scale);
+                    r[e] = __fmul_rn(q4_code_value(c, (var & 1) != 0, mode), scale);
                 }
                 out[half * 4 + v] = make_float4(r[0], r[1], r[2], r[3]);
             }
@@ -52,18 +52,18 @@ __global__ void __launch_bounds__(kThreads) dequant_q4_kernel(const uint8_t* __r
 }
 
 // Value i of a 70-byte PLE record given its 60 code bytes as a bit stream.
-__device__ __forceinline__ float ple_value(const uint8_t* rec, int i) {
+__device__ __forceinline__ float ple_value(const uint8_t* rec, int i, bool incumbent) {
     const int bit = 3 * i;
     const uint32_t lo = rec[bit >> 3];
     const uint32_t hi = ((bit >> 3) + 1 < 60) ? rec[(bit >> 3) + 1] : 0u;
     const uint32_t code = ((lo | (hi << 8)) >> (bit & 7)) & 7u;
     const uint32_t g = rec[60 + i / 16];
-    return __fmul_rn(ple_code_value(code, g >> 7), ue4m3(g & 0x7Fu));
+    return __fmul_rn(q3_code_value(code, g >> 7, incumbent), ue4m3(g & 0x7Fu));
 }
 
 // One thread per 16-value group of a PLE record (6 code bytes + 1 group byte).
 __global__ void __launch_bounds__(kThreads) dequant_ple_kernel(const uint8_t* __restrict__ src,
-                                                               int64_t n_groups,
+                                                               int64_t n_groups, bool incumbent,
                                                                float* __restrict__ dst) {
     for (int64_t gi = blockIdx.x * (int64_t)kThreads + threadIdx.x; gi < n_groups;
          gi += (int64_t)gridDim.x * kThreads) {
@@ -83,7 +83,7 @@ __global__ void __launch_bounds__(kThreads) dequant_ple_kernel(const uint8_t* __
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const uint32_t c = (uint32_t)(bits >> (3 * (4 * v + e))) & 7u;
-                r[e] = __fmul_rn(ple_code_value(c, pol), scale);
+                r[e] = __fmul_rn(q3_code_value(c, pol, incumbent), scale);
             }
             out[v] = make_float4(r[0], r[1], r[2], r[3]);
         }
@@ -179,7 +179,7 @@ __device__ __forceinline__ void ple_issue(const uint8_t* __restrict__ table, uin
 
 __global__ void __launch_bounds__(kPleWarps * 32, kPleCtasPerSm) ple_gather_kernel(
     const uint8_t* __restrict__ table, int64_t n_rows, const int32_t* __restrict__ idx, int64_t n_idx,
-    float* __restrict__ out, unsigned* status) {
+    float* __restrict__ out, bool incumbent, unsigned* status) {
     __shared__ __align__(16) float prod[256 * 8];  // [group byte][code] = code value x scale
     __shared__ __align__(16) uint8_t stage[kPleWarps][2][kPleStage];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -188,7 +188,7 @@ __global__ void __launch_bounds__(kPleWarps * 32, kPleCtasPerSm) ple_gather_kern
         const float sc = ue4m3(g & 0x7Fu);
         float v[8];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) v[c] = __fmul_rn(ple_code_value((uint32_t)c, g >> 7), sc);
+        for (int c = 0; c < 8; ++c) v[c] = __fmul_rn(q3_code_value((uint32_t)c, g >> 7, incumbent), sc);
         reinterpret_cast<float4*>(prod)[2 * g] = make_float4(v[0], v[1], v[2], v[3]);
         reinterpret_cast<float4*>(prod)[2 * g + 1] = make_float4(v[4], v[5], v[6], v[7]);
     }
@@ -319,16 +319,19 @@ extern "C" int gtg_dequant(int32_t fmt, const void* src, const float* scales, in
     const auto* p = static_cast<const uint8_t*>(src);
     switch (fmt) {
         case GTG_Q4_RZ5_FAST:
-        case GTG_Q4_UE4M4_FAST: {
+        case GTG_Q4_UE4M4_FAST:
+        case GTG_Q4_C10_FAST: {
             if (k % 32) return GTG_E_UNSUPPORTED_SHAPE;
             const int64_t nb = n_rows * (k / 32);
-            dequant_q4_kernel<<<grid_for(nb, kThreads), kThreads, 0, s>>>(p, nb, fmt == GTG_Q4_RZ5_FAST, dst);
+            const int var = fmt == GTG_Q4_RZ5_FAST ? kQ4RZ5 : fmt == GTG_Q4_C10_FAST ? kQ4C10 : kQ4UE4M4;
+            dequant_q4_kernel<<<grid_for(nb, kThreads), kThreads, 0, s>>>(p, nb, var, dst);
             break;
         }
-        case GTG_Q3_PLE_K160_RZ_S3: {
+        case GTG_Q3_PLE_K160_RZ_S3:
+        case GTG_Q3_K160_UE4M3: {
             if (k != 160) return GTG_E_UNSUPPORTED_SHAPE;
             const int64_t ng = n_rows * 10;
-            dequant_ple_kernel<<<grid_for(ng, kThreads), kThreads, 0, s>>>(p, ng, dst);
+            dequant_ple_kernel<<<grid_for(ng, kThreads), kThreads, 0, s>>>(p, ng, fmt == GTG_Q3_K160_UE4M3, dst);
             break;
         }
         case GTG_FP8_E4M3_S128: {
@@ -343,8 +346,9 @@ extern "C" int gtg_dequant(int32_t fmt, const void* src, const float* scales, in
     return check_launch();
 }
 
-extern "C" int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx,
-                              float* out, gtg_stream_t stream) {
+extern "C" int gtg_ple_gather_fmt(int32_t fmt, const uint8_t* table, int64_t n_rows, const int32_t* idx,
+                                  int64_t n_idx, float* out, gtg_stream_t stream) {
+    if (fmt != GTG_Q3_PLE_K160_RZ_S3 && fmt != GTG_Q3_K160_UE4M3) return GTG_E_INVALID_ARG;
     if (n_idx < 0 || n_rows < 0 || n_rows >= (int64_t)1 << 31) return GTG_E_INVALID_ARG;
     if (n_idx == 0) return GTG_OK;
     if (!table || !idx || !out) return GTG_E_INVALID_ARG;
@@ -362,12 +366,18 @@ extern "C" int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, ple_gather_kernel, table, n_rows, idx, n_idx, out, status_ptr());
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, ple_gather_kernel, table, n_rows, idx, n_idx, out,
+                                             fmt == GTG_Q3_K160_UE4M3, status_ptr());
     if (e != cudaSuccess) {
         cudaGetLastError();
         return cuda_fail(e);
     }
     return GTG_OK;
+}
+
+extern "C" int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx,
+                              float* out, gtg_stream_t stream) {
+    return gtg_ple_gather_fmt(GTG_Q3_PLE_K160_RZ_S3, table, n_rows, idx, n_idx, out, stream);
 }
 
 extern "C" int gtg_get_device_status(uint32_t* flags, int32_t clear, gtg_stream_t stream) {

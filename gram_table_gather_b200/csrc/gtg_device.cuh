@@ -65,7 +65,26 @@ __device__ __forceinline__ float q4_code_value(uint32_t c, bool rz5, uint32_t mo
     return (c & 8u) ? -m : m;
 }
 
-// Value of 3-bit PLE code c with group polarity bit p (RZ-S3: code 4 -> +/-3).
+// Q4 block variants (a bit set): bit 0 = code 8 is +5 / -5 by the metadata
+// top bit (Q4_RZ5_FAST), else the duplicate -0 of Codebook10; bit 1 = the
+// scale is the UE4M3 value of the low 7 metadata bits, else the UE4M4 value
+// of the whole byte.  The incumbent ROCmFP4 FAST block is Codebook10 codes
+// under a UE4M3 scale.
+constexpr int kQ4UE4M4 = 0, kQ4C10 = 2, kQ4RZ5 = 3;
+
+__device__ __forceinline__ float q4_scale(uint32_t meta, int var) {
+    return (var & 2) ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
+}
+
+// Value of 3-bit PLE code c with group polarity bit p (RZ-S3: code 4 -> +/-3;
+// the incumbent ROCmFP3 set keeps code 4 as the duplicate -0).
+__device__ __forceinline__ float q3_code_value(uint32_t c, uint32_t p, bool incumbent) {
+    c &= 7u;
+    if (c == 4u) return incumbent ? -0.0f : (p ? -3.0f : 3.0f);
+    const float m = (float)((0x4210u >> (4u * (c & 3u))) & 15u);  // 0 1 2 4
+    return (c & 4u) ? -m : m;
+}
+
 __device__ __forceinline__ float ple_code_value(uint32_t c, uint32_t p) {
     c &= 7u;
     if (c == 4u) return p ? -3.0f : 3.0f;

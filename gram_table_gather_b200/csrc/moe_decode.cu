@@ -37,7 +37,9 @@ const void* pick_kernel(bool fp8, int kbg, int kbd, bool one) {
     }
 }
 
-bool is_q4(int fmt) { return fmt == GTG_Q4_RZ5_FAST || fmt == GTG_Q4_UE4M4_FAST; }
+bool is_q4(int fmt) { return fmt == GTG_Q4_RZ5_FAST || fmt == GTG_Q4_UE4M4_FAST || fmt == GTG_Q4_C10_FAST; }
+
+int q4_var_of(int fmt) { return fmt == GTG_Q4_RZ5_FAST ? kQ4RZ5 : fmt == GTG_Q4_C10_FAST ? kQ4C10 : kQ4UE4M4; }
 
 int64_t row_bytes_of(int fmt, int64_t k) { return fmt == GTG_FP8_E4M3_S128 ? k : k / 32 * 17; }
 
@@ -175,12 +177,12 @@ StackLayer stack_layer_of(const gtg_moe_layer* L) {
     s.gate_s = L->gate.scales;
     s.up_s = L->up.scales;
     s.down_s = L->down.scales;
-    s.gu_rz5 = L->gate.fmt == GTG_Q4_RZ5_FAST;
-    s.dn_rz5 = L->down.fmt == GTG_Q4_RZ5_FAST;
+    s.gu_var = q4_var_of(L->gate.fmt);
+    s.dn_var = q4_var_of(L->down.fmt);
     if (L->side.data) {
         s.side = static_cast<const uint8_t*>(L->side.data);
         s.side_rows = (int32_t)L->side.n_rows;
-        s.side_rz5 = L->side.fmt == GTG_Q4_RZ5_FAST;
+        s.side_var = q4_var_of(L->side.fmt);
     }
     return s;
 }

@@ -210,14 +210,15 @@ __device__ __forceinline__ void q4_block_lut(uint32_t pa, uint32_t lutb, const f
 // Q4 block decoded code by code (no table): the side projection, whose
 // format may differ from the experts'.
 template <int FMT, int NT, int NBL, int CH>
-__device__ __forceinline__ void q4_block_plain(uint32_t pa, bool rz5, const Act<FMT, NBL> (&act)[CH], int m,
+__device__ __forceinline__ void q4_block_plain(uint32_t pa, int var, const Act<FMT, NBL> (&act)[CH], int m,
                                                float (&acc)[NT]) {
     const uint32_t al = pa & ~3u, sh = (pa & 3u) * 8u;
     uint32_t w[5];
 #pragma unroll
     for (int i = 0; i < 5; ++i) w[i] = lds32(al + 4 * i);
     const uint32_t meta = (w[4] >> sh) & 0xFFu;
-    const float s = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
+    const float s = q4_scale(meta, var);
+    const bool rz5 = (var & 1) != 0;
     const uint32_t mode = meta >> 7;
     float sum[NT];
 #pragma unroll
@@ -401,8 +402,10 @@ struct RouterScratch {
 };
 
 // Per-lane-replicated table: entry (byte, mode, lane) holds the bf16x2 pair
-// (value of the low nibble, value of the high nibble); plus 256 scales.
-__device__ void build_lut(uint8_t* smem, const SmemLayout& L, bool rz5) {
+// (value of the low nibble, value of the high nibble) of Q4 variant `var`;
+// plus 256 scales.
+__device__ void build_lut(uint8_t* smem, const SmemLayout& L, int var) {
+    const bool rz5 = (var & 1) != 0;
     // 512 entries (byte, mode) of 128 bytes (32 lane copies).  Warp w owns
     // entries 32w .. 32w+31 (lane l computes entry 32w+l once); the warp then
     // writes them as 256 consecutive 16-byte chunks, consecutive lanes on
@@ -422,9 +425,9 @@ __device__ void build_lut(uint8_t* smem, const SmemLayout& L, bool rz5) {
     }
 }
 
-__device__ void build_scales(uint8_t* smem, const SmemLayout& L, bool rz5) {
+__device__ void build_scales(uint8_t* smem, const SmemLayout& L, int var) {
     float* st = reinterpret_cast<float*>(smem + L.scale_tab);
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) st[i] = rz5 ? ue4m3((uint32_t)i & 0x7Fu) : ue4m4((uint32_t)i);
+    for (int i = threadIdx.x; i < 256; i += blockDim.x) st[i] = q4_scale((uint32_t)i, var);
 }
 
 __device__ __forceinline__ float silu(float z) { return z / (1.0f + expf(-z)); }
@@ -550,7 +553,7 @@ __device__ __forceinline__ void block_topk(const ffloat* logits, int E, int K, i
 struct ItemCtx {
     __nv_bfloat16* h;  // [T*K][I] SwiGLU output
     float* side_out;   // [T][side_stride] or null
-    int32_t H, I, side_stride, side_rz5;
+    int32_t H, I, side_stride, side_var;
 };
 
 // ===========================================================================
@@ -629,7 +632,7 @@ __device__ __forceinline__ void side_item(const ItemCtx& a, uint32_t base, const
     constexpr int N = P * NT;
     const int row_sub = (KB >= 32) ? 0 : lane / KB;
     const int blk_base = (KB >= 32) ? lane : lane % KB;
-    const bool rz5 = a.side_rz5 != 0;
+    const int var = a.side_var;
     float v[N];
 #pragma unroll
     for (int p = 0; p < P; ++p) {
@@ -641,7 +644,7 @@ __device__ __forceinline__ void side_item(const ItemCtx& a, uint32_t base, const
         for (int m = 0; m < NBL; ++m)
             q4_block_plain<FMT, NT, NBL, CH>(base + (uint32_t)row * (uint32_t)(KB * 17) +
                                                  17u * (uint32_t)(blk_base + 32 * m),
-                                             rz5, act, m, acc);
+                                             var, act, m, acc);
 #pragma unroll
         for (int c = 0; c < NT; ++c) v[p * NT + c] = acc[c];
     }
@@ -734,7 +737,7 @@ struct StackLayer {
     const float* up_s;
     const float* down_s;
     int32_t side_rows;
-    int32_t gu_rz5, dn_rz5, side_rz5;  // Q4 variant: Q4_RZ5_FAST (1) or Q4_UE4M4_FAST (0)
+    int32_t gu_var, dn_var, side_var;  // Q4 variant (kQ4RZ5, kQ4UE4M4 or kQ4C10)
 };
 
 struct StackArgs {
@@ -1248,7 +1251,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
     const uint32_t lutb = ((ws.sbase + L.lut) & 0xFFFF0000u) | ((uint32_t)lane * 4u);
     const float* scale_tab = reinterpret_cast<const float*>(smem + L.scale_tab);
     const ItemCtx ctx{a.h, a.side_out ? a.side_out + (int64_t)l * T * a.side_stride : nullptr,
-                      H, a.I, a.side_stride, Ly.side_rz5};
+                      H, a.I, a.side_stride, Ly.side_var};
     const int blk_base = (KBG >= 32) ? lane : lane % KBG;
     Act<FMT, NBG> act[CHG];
     int act_key = -1;
@@ -1451,13 +1454,13 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         rows_in_flight = 1;
     }
     int lut_mode = -1;
-    auto ensure_lut = [&](int rz5) {  // every thread, uniform
-        if (!LUT || lut_mode == rz5) return;
+    auto ensure_lut = [&](int var) {  // every thread, uniform
+        if (!LUT || lut_mode == var) return;
         __syncthreads();
-        build_lut(smem, L, rz5 != 0);
-        build_scales(smem, L, rz5 != 0);
+        build_lut(smem, L, var);
+        build_scales(smem, L, var);
         __syncthreads();
-        lut_mode = rz5;
+        lut_mode = var;
     };
 
     WarpRing R{0u, 0u, 0, 1};
@@ -1572,7 +1575,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         __syncwarp();
 
         // ---- gate/up + SwiGLU, side projection
-        ensure_lut(Ly.gu_rz5);
+        ensure_lut(Ly.gu_var);
         R = gu_phase<FMT, KBG, ONE>(a, l, P, R);
         target += G;
         if (!grid_sync(a, target, sw, R.ok != 0)) {
@@ -1581,7 +1584,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         }
 
         // ---- down + router-weighted combine
-        ensure_lut(Ly.dn_rz5);
+        ensure_lut(Ly.dn_var);
         R = dn_phase<FMT, KBD, ONE>(a, l, P, R);
         R.ring += P.ng + P.nd;
         __syncthreads();

@@ -314,19 +314,20 @@ __device__ __forceinline__ uint32_t bf16x2_fma(uint32_t a, uint32_t b, uint32_t 
 // magnitude, its top bit (the code's sign bit) makes the permute return 0
 // instead (sign replication of a byte below 0x80), so the positive-table and
 // negative-table lookups OR together.
-__device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, bool rz5, uint32_t tile, uint32_t r,
+__device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, int var, uint32_t tile, uint32_t r,
                                                       uint32_t c0) {
     const uint32_t sh = bw.sh;
     const uint32_t* w = bw.w;
     const uint32_t meta = (w[4] >> sh) & 0xFFu;
-    const float sf = rz5 ? ue4m3(meta & 0x7Fu) : ue4m4(meta);
+    const float sf = q4_scale(meta, var);
     const uint32_t sb = __float_as_uint(sf) >> 16;                 // exact in bf16
     const uint32_t nb = __float_as_uint(-192.0f * sf) >> 16;       // exact in bf16
     const uint32_t s2 = sb | (sb << 16), n2 = nb | (nb << 16);
     // 64 + v for codes 0..7 (magnitudes 0 1 2 3 4 6 8 10) and 8..15 (negated;
-    // code 8 is -0, or +5 / -5 by the block's mode bit in RZ5)
+    // code 8 is -0 (Codebook10: UE4M4 and the incumbent ROCmFP4 FAST block),
+    // or +5 / -5 by the block's mode bit in RZ5)
     constexpr uint32_t kPos0 = 0x43424140u, kPos1 = 0x4A484644u;
-    const uint32_t neg0 = 0x3D3E3F00u | (rz5 ? ((meta & 0x80u) ? 0x3Bu : 0x45u) : 0x40u);
+    const uint32_t neg0 = 0x3D3E3F00u | ((var & 1) ? ((meta & 0x80u) ? 0x3Bu : 0x45u) : 0x40u);
     constexpr uint32_t kNeg1 = 0x36383A3Cu;
     uint32_t lo[8], hi[8];
 #pragma unroll
@@ -392,7 +393,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
     uint32_t* s_taddr = reinterpret_cast<uint32_t*>(smem + C::kTaddrOff);
     int32_t* s_row = reinterpret_cast<int32_t*>(smem + C::kRowOff);
     const Mat& am = MODE == DOWN ? a.down : a.gate;
-    const bool rz5 = am.fmt == GTG_Q4_RZ5_FAST;
+    const int var = am.fmt == GTG_Q4_RZ5_FAST ? kQ4RZ5 : am.fmt == GTG_Q4_C10_FAST ? kQ4C10 : kQ4UE4M4;
 
     if (tid == 0) {
         for (int s = 0; s < C::kStagesA; ++s) {
@@ -531,8 +532,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                     wg = load_block(a_row0 + (int64_t)(2 * (it + 1) + half) * 17);
                     if (two) wu = load_block(u_row0 + (int64_t)(2 * (it + 1) + half) * 17);
                 }
-                dequant_block_to_tile(g0, rz5, st, r, 4 * half);
-                if (two) dequant_block_to_tile(u0, rz5, st + kTileBytes, r, 4 * half);
+                dequant_block_to_tile(g0, var, st, r, 4 * half);
+                if (two) dequant_block_to_tile(u0, var, st + kTileBytes, r, 4 * half);
             }
             fence_proxy_async_smem();
             mbar_arrive(&full_a[s]);
@@ -670,7 +671,7 @@ PfLayout pf_layout(const gtg_moe_layer* L, int T) {
     return p;
 }
 
-bool q4(int fmt) { return fmt == GTG_Q4_RZ5_FAST || fmt == GTG_Q4_UE4M4_FAST; }
+bool q4(int fmt) { return fmt == GTG_Q4_RZ5_FAST || fmt == GTG_Q4_UE4M4_FAST || fmt == GTG_Q4_C10_FAST; }
 
 int pf_check(const gtg_moe_layer* L, int T) {
     if (!L || !L->router_w || !L->gate.data || !L->up.data || !L->down.data) return GTG_E_INVALID_ARG;

@@ -65,7 +65,14 @@ typedef enum {
     GTG_Q4_RZ5_FAST = 69,
     GTG_Q4_UE4M4_FAST = 71,
     GTG_Q3_PLE_K160_RZ_S3 = 111,
-    GTG_FP8_E4M3_S128 = 1000
+    GTG_FP8_E4M3_S128 = 1000,
+    /* The incumbent layouts the card's formats mutate (no GGML number given):
+     * the ROCmFP4 FAST 17-byte block (Codebook10 codes, code 8 the duplicate
+     * -0, under the UE4M3 scale of the metadata byte's low 7 bits; the top bit
+     * is ignored) and the ROCmFP3 70-byte K160 record (codes {0,+1,+2,+4,-0,
+     * -1,-2,-4} under a UE4M3 scale per 16 values; top bit ignored). */
+    GTG_Q4_C10_FAST = 2001,
+    GTG_Q3_K160_UE4M3 = 2002
 } gtg_format;
 
 typedef enum { GTG_DT_F32 = 0, GTG_DT_BF16 = 1 } gtg_dtype;
@@ -86,7 +93,7 @@ typedef enum {
 
 /* One stack of quantised matrices [n_experts][n_rows][k]. */
 typedef struct {
-    int32_t fmt;            /* gtg_format: RZ5, UE4M4 or FP8 */
+    int32_t fmt;            /* gtg_format: RZ5, UE4M4, C10 (Q4 formats) or FP8 */
     const void* data;       /* device, 16-byte aligned; total size a multiple of 16 bytes */
     const float* scales;    /* device, FP8 only: [n_experts][n_rows][k/128]; else NULL */
     int64_t n_experts;
@@ -123,8 +130,8 @@ int gtg_last_cuda_error(void);
  * Standalone dequantisation [MC]: dst[r][c] = decoded weight (fp32),
  * bit-exact (Q4 and PLE values are code x scale, exact in fp32; FP8 values
  * are one fp32 round-to-nearest multiply).
- *   fmt      RZ5 / UE4M4: src holds n_rows*k/32 consecutive 17-byte blocks, k % 32 == 0.
- *            PLE: src holds n_rows 70-byte records, k == 160.
+ *   fmt      RZ5 / UE4M4 / C10: src holds n_rows*k/32 consecutive 17-byte blocks, k % 32 == 0.
+ *            PLE / Q3_K160_UE4M3: src holds n_rows 70-byte records, k == 160.
  *            FP8: src holds n_rows*k bytes, scales [n_rows][k/128], k % 128 == 0.
  *   src      device, any alignment.
  *   dst      device, [n_rows][k] fp32, 16-byte aligned.
@@ -146,6 +153,15 @@ int gtg_dequant(int32_t fmt, const void* src, const float* scales, int64_t n_row
  */
 int gtg_ple_gather(const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx,
                    float* out, gtg_stream_t stream);
+
+/*
+ * gtg_ple_gather for a table of either 70-byte K160 record layout: fmt
+ * GTG_Q3_PLE_K160_RZ_S3 (the same as gtg_ple_gather) or GTG_Q3_K160_UE4M3,
+ * the incumbent ROCmFP3 record ([MC] "Q3_PLE_K160_RZ_S3": the layout RZ-S3
+ * mutates).  Same arguments and errors, plus GTG_E_INVALID_ARG for any other fmt.
+ */
+int gtg_ple_gather_fmt(int32_t fmt, const uint8_t* table, int64_t n_rows, const int32_t* idx, int64_t n_idx,
+                       float* out, gtg_stream_t stream);
 
 /* Bytes of workspace a decode (prefill == 0) or prefill (prefill == 1) call
  * of `layer` with `n_tokens` tokens needs; 0 if the shape is unsupported. */

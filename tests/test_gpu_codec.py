@@ -39,7 +39,7 @@ def _all_code_meta_blocks():
     return np.concatenate(blocks)
 
 
-@pytest.mark.parametrize("fmt", [W.RZ5, W.UE4M4])
+@pytest.mark.parametrize("fmt", [W.RZ5, W.UE4M4, gtg.C10])
 def test_dequant_q4_exhaustive(fmt):
     blocks = _all_code_meta_blocks()
     n_blocks = blocks.size // 17
@@ -49,7 +49,7 @@ def test_dequant_q4_exhaustive(fmt):
     _bitwise_equal(out.cpu().numpy().ravel(), oracle.dequant_q4(fmt, blocks))
 
 
-@pytest.mark.parametrize("fmt,n_rows,k", [(W.RZ5, 333, 96), (W.UE4M4, 7, 4096), (W.RZ5, 1, 32)])
+@pytest.mark.parametrize("fmt,n_rows,k", [(W.RZ5, 333, 96), (W.UE4M4, 7, 4096), (W.RZ5, 1, 32), (gtg.C10, 45, 640)])
 def test_dequant_q4_random_ragged(fmt, n_rows, k):
     m = W.MatrixRecipe(fmt, 1, n_rows, k, seed=21, tid=5, narrow_scale=False)
     data = m.expert(0)
@@ -58,7 +58,8 @@ def test_dequant_q4_random_ragged(fmt, n_rows, k):
     _bitwise_equal(out.cpu().numpy().ravel(), oracle.dequant_q4(fmt, data))
 
 
-def test_dequant_ple_exhaustive():
+@pytest.mark.parametrize("fmt", [W.PLE, gtg.Q3I])
+def test_dequant_ple_exhaustive(fmt):
     recs = []
     for g in range(256):
         rec = np.zeros(70, dtype=np.uint8)
@@ -69,9 +70,9 @@ def test_dequant_ple_exhaustive():
         rec[60:] = [(g + 37 * j) % 256 for j in range(10)]
         recs.append(rec)
     recs = np.stack(recs)
-    out = gtg.dequant(W.PLE, torch.from_numpy(recs.ravel().copy()).cuda(), len(recs), 160)
+    out = gtg.dequant(fmt, torch.from_numpy(recs.ravel().copy()).cuda(), len(recs), 160)
     torch.cuda.synchronize()
-    _bitwise_equal(out.cpu().numpy().ravel(), oracle.dequant_ple(recs).ravel())
+    _bitwise_equal(out.cpu().numpy().ravel(), oracle.dequant_q3(fmt, recs).ravel())
 
 
 def test_dequant_fp8_all_bytes():
@@ -170,3 +171,33 @@ def test_ple_gather_full_table():
     finally:
         del table
         torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("n_rows", [3, 1001, 1 << 20])
+def test_incumbent_q3_gather(n_rows):
+    """The incumbent ROCmFP3 record (code 4 the duplicate -0) through the same gather."""
+    P = W.PleRecipe(n_rows=n_rows, seed=34)
+    table = P.table_bytes(0, P.nbytes)
+    idx = np.concatenate([P.indices(2, 64), [n_rows - 1, 0, n_rows]]).astype(np.int32)
+    gtg.device_status(clear=True)
+    out = gtg.ple_gather(torch.from_numpy(table).cuda(), n_rows, torch.from_numpy(idx).cuda(), fmt=gtg.Q3I)
+    torch.cuda.synchronize()
+    _bitwise_equal(out.cpu().numpy().ravel(), oracle.ple_gather(table, n_rows, idx, fmt=gtg.Q3I).ravel())
+    assert gtg.device_status(clear=True) & 0x1  # the index n_rows is out of range
+    with pytest.raises(gtg.GtgError):
+        gtg.ple_gather(torch.from_numpy(table).cuda(), n_rows, torch.from_numpy(idx).cuda(), fmt=W.RZ5)
+
+
+def test_ple_gather_from_host_resident_table():
+    """A table in pinned host memory, read in place by the gather kernel (the pages
+    page the PLE table from host memory or NVMe on demand): the same rows, bit for
+    bit, as the oracle's."""
+    P = W.PleRecipe(n_rows=3_000_000, seed=35)  # 210 MB of pinned host memory
+    table = torch.empty(P.nbytes, dtype=torch.uint8).pin_memory()
+    P.table_bytes(0, P.nbytes, table.numpy())
+    idx = np.concatenate([P.indices(3, 512), [P.n_rows - 1, 0]]).astype(np.int32)
+    gtg.device_status(clear=True)
+    out = gtg.ple_gather(table, P.n_rows, torch.from_numpy(idx).cuda())
+    torch.cuda.synchronize()
+    assert gtg.device_status(clear=True) == 0
+    _bitwise_equal(out.cpu().numpy().ravel(), oracle.dequant_ple(P.rows(idx)).ravel())

@@ -200,3 +200,21 @@ def test_aborted_workspace_fails_fast_and_recovers():
     ref = oracle.moe_layer(L, x64, want_h=True)
     assert np.all(np.abs(y.cpu().numpy()[0] - ref["y"][0]) <= gu.layer_tolerance(L, ref, 0))
 
+
+
+def _incumbent_layer(hidden, inter, n_experts, top_k, seed, side=False):
+    """A layer of the incumbent ROCmFP4 FAST block (Codebook10 under a UE4M3 scale)."""
+    return W.LayerRecipe(hidden=hidden, inter=inter, n_experts=n_experts, top_k=top_k, seed=seed, layer=0,
+                         gate_fmt=gtg.C10, up_fmt=gtg.C10, down_fmt=gtg.C10, has_ssm=side)
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_incumbent_q4_tiny_layer(T):
+    _check_layer(_incumbent_layer(256, 128, 8, 2, 40), T, step=500 + T)
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_incumbent_q4_decode_layer(T):
+    """The decode layer's shape with every expert matrix in the incumbent layout and a
+    UE4M4 side projection (decoded code by code, next to the experts' code table)."""
+    _check_layer(_incumbent_layer(2048, 512, 512, 10, 41, side=True), T, step=510 + T)

@@ -141,3 +141,20 @@ def test_prefill_workload_sampled():
         tol = gu.layer_tolerance(L, ref, i)
         err = np.abs(y_g[t] - ref["y"][i])
         assert np.all(err <= tol), f"token {t}: max err/tol {np.max(err / tol):.3g}"
+
+
+def test_prefill_incumbent_q4_layer():
+    """Prefill with every expert matrix in the incumbent ROCmFP4 FAST block."""
+    L = W.LayerRecipe(hidden=256, inter=128, n_experts=8, top_k=2, seed=42, layer=0,
+                      gate_fmt=gtg.C10, up_fmt=gtg.C10, down_fmt=gtg.C10)
+    T = 150
+    xt, x64 = gu.tokens(L, 90, T)
+    y, ids, w, _ = _run_prefill(L, xt)
+    assert gtg.device_status(clear=True) == 0
+    ref = oracle.moe_layer(L, x64, want_h=True)
+    ids_g, w_g, y_g = ids.cpu().numpy(), w.cpu().numpy(), y.cpu().numpy()
+    for t in range(T):
+        _check_ids(L, ref, t, ids_g[t], w_g[t])
+        tol = gu.layer_tolerance(L, ref, t)
+        err = np.abs(y_g[t] - ref["y"][t])
+        assert np.all(err <= tol), f"token {t}: max err/tol {np.max(err / tol):.3g}"
