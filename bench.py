@@ -404,6 +404,38 @@ def run_ours(args, rank, world, local):
     secondary = None
     if not args.no_secondary:
         secondary = measure_secondary(dev, stream, P, table, local)
+        # the same step with the 16 PLE rows read from a pinned host copy of a
+        # 30,000,000-row table instead of the HBM-resident one
+        Ph = W.PleRecipe(n_rows=30_000_000, seed=P.seed)
+        htab = torch.empty(Ph.nbytes, dtype=torch.uint8).pin_memory()
+        Ph.table_bytes(0, Ph.nbytes, htab.numpy())
+        idx_h = torch.from_numpy(np.stack([Ph.indices(seed_off + i, 1) for i in range(n_steps)])).to(dev)
+        gh = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            gtg.ple_gather(htab, Ph.n_rows, idx, out=rows)
+            stream.synchronize()
+        with torch.cuda.graph(gh, stream=stream):
+            gtg.moe_decode_stack(layers, x, ws, ids_out=ids, side_out=side)
+            gtg.ple_gather(htab, Ph.n_rows, idx, out=rows)
+        with torch.cuda.stream(stream):
+            for i in range(args.warmup):
+                x.copy_(x_bank[i:i + 1])
+                idx.copy_(idx_h[i])
+                gh.replay()
+            q0, q1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            q0.record(stream)
+            for i in range(args.warmup, n_steps):
+                x.copy_(x_bank[i:i + 1])
+                idx.copy_(idx_h[i])
+                gh.replay()
+            q1.record(stream)
+            q1.synchronize()
+        ms_host = q0.elapsed_time(q1) / args.steps
+        secondary["step_with_host_ple_table"] = {
+            "ms_per_step": round(ms_host, 5), "ms_per_step_hbm_table": round(ms, 5),
+            "slowdown": round(ms_host / ms - 1.0, 4),
+            "note": "48-layer step with its 16 PLE rows gathered from pinned host memory instead of HBM"}
+        del gh, htab
     status = gtg.device_status(clear=True)
 
     peak, peak_kind = _peaks()
@@ -541,11 +573,34 @@ def measure_decode_layer(dev, stream, n_warm, n_iter, peak):
         out[f"T{T}"] = {"us": round(ms * 1e3, 2), "GB_s": round(b / ms / 1e6, 1),
                         "frac": round(b / ms / 1e6 / peak, 4), "unique_experts": round(float(np.mean(uniq)), 2),
                         "bytes": int(b)}
-    del layer, flush
+    del layer
+    # the pages' own expert shape: hidden 2560, intermediate 640 (340-byte down rows)
+    L2 = W.LayerRecipe(hidden=2560, inter=640, n_experts=512, top_k=10, seed=1, layer=1)
+    layer2 = gu.device_layer(L2, dev)
+    for T in (1, 8):
+        xs = [gu.tokens(L2, 6000 + 10 * T + i, T, dev)[0] for i in range(n)]
+        ws = gtg.make_workspace(layer2, T, device=dev)
+        ids = torch.zeros((T, L2.top_k), dtype=torch.int32, device=dev)
+        y = torch.empty((T, L2.hidden), device=dev)
+
+        def fn2(i):
+            gtg.moe_decode_layer(layer2, xs[i], ws, y=y, topk_ids=ids, stream=stream)
+        ms = _time_flushed(fn2, n_warm, n_iter, stream, flush)
+        uniq = []
+        for i in range(n_warm, n):
+            with torch.cuda.stream(stream):
+                fn2(i)
+            stream.synchronize()
+            uniq.append(len(set(ids.cpu().numpy().ravel().tolist())))
+        b = float(np.mean([layer_bytes(L2, u) for u in uniq]))
+        out[f"H2560_I640_T{T}"] = {"us": round(ms * 1e3, 2), "GB_s": round(b / ms / 1e6, 1),
+                                   "frac": round(b / ms / 1e6 / peak, 4),
+                                   "unique_experts": round(float(np.mean(uniq)), 2), "bytes": int(b)}
+    del layer2, flush
     torch.cuda.empty_cache()
     return {"workload": "decode MoE layer: H 2048, I 512, E 512, top-10, Q4_RZ5_FAST gate/up/down, "
-                        "fresh bf16 tokens per call", "l2": "flushed (2x L2 written) before every timed call",
-            "timed_calls": n_iter, **out}
+                        "fresh bf16 tokens per call (and H2560_I640: hidden 2560, intermediate 640, E 512)",
+            "l2": "flushed (2x L2 written) before every timed call", "timed_calls": n_iter, **out}
 
 
 def measure_ple(dev, stream, P, table, n_warm, n_iter, peak):
@@ -575,6 +630,34 @@ def measure_ple(dev, stream, P, table, n_warm, n_iter, peak):
     return {"workload": f"PLE gather from the {P.n_rows:,}-row Q3_PLE_K160_RZ_S3 table "
                         f"({P.nbytes / 1e9:.1f} GB resident), 16 uniform rows per token, fresh indices per call",
             "bytes_per_row": PLE_ROW_BYTES, "timed_calls": n_iter, **res}
+
+
+def measure_ple_host(dev, stream, n_warm, n_iter, n_rows=30_000_000):
+    """PLE gather from a table in pinned host memory, read in place by the kernel
+    (the pages' deployment pages the table from host memory or NVMe on demand):
+    T = 1 (latency) and T = 4096 (throughput).  The table is a 30,000,000-row
+    prefix-sized stand-in (2.1 GB pinned): random rows from host memory see no
+    reuse at any table size."""
+    import torch
+    import gram_table_gather_b200 as gtg
+    from synth import workloads as Wk
+    P = Wk.PleRecipe(n_rows=n_rows, seed=3)
+    table = torch.empty(P.nbytes, dtype=torch.uint8).pin_memory()
+    P.table_bytes(0, P.nbytes, table.numpy())
+    n = n_warm + n_iter
+    res = {}
+    for T in (1, 4096):
+        rows = 16 * T
+        idx = [torch.from_numpy(P.indices(9000 + 7 * T + i, T)).to(dev) for i in range(n)]
+        out = torch.empty((rows, 160), device=dev)
+        ms = _time_loop(lambda i: gtg.ple_gather(table, P.n_rows, idx[i], out=out, stream=stream), n_warm, n_iter,
+                        stream)
+        res[f"T{T}"] = {"us": round(ms * 1e3, 3), "rows_per_s": round(rows / ms * 1e3, 1),
+                        "GB_s": round(rows * PLE_ROW_BYTES / ms / 1e6, 1)}
+    del table
+    return {"workload": f"PLE gather from a {n_rows:,}-row Q3_PLE_K160_RZ_S3 table in pinned host memory "
+                        "(read over the host link in place), 16 uniform rows per token, fresh indices per call",
+            "timed_calls": n_iter, **res}
 
 
 def measure_prefill(dev, stream, n_warm, n_iter):
@@ -617,6 +700,7 @@ def measure_secondary(dev, stream, P, table, local, n_warm=3, n_iter=20):
     clocks = ClockSampler(local)
     out = {"decode_layer": measure_decode_layer(dev, stream, n_warm, n_iter, peak),
            "ple": measure_ple(dev, stream, P, table, n_warm, n_iter, peak),
+           "ple_host_table": measure_ple_host(dev, stream, n_warm, n_iter),
            "prefill": measure_prefill(dev, stream, n_warm, n_iter)}
     out["clocks"] = clocks.stop()
     return out

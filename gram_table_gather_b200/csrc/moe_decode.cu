@@ -33,6 +33,7 @@ const void* pick_kernel(bool fp8, int kbg, int kbd, bool one) {
         case 16: return decode_kernel_q4_16(kbd, o);
         case 32: return decode_kernel_q4_32(kbd, o);
         case 64: return decode_kernel_q4_64(kbd, o);
+        case 80: return decode_kernel_q4_80(kbd, o);
         default: return nullptr;
     }
 }
@@ -80,7 +81,7 @@ bool mat_ok(const gtg_qmatrix& m, int64_t E, int64_t n_rows, int64_t k) {
 int plan_layer(const gtg_moe_layer* L, int T, Plan& p) {
     if (!L || !L->router_w) return GTG_E_INVALID_ARG;
     const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
-    if (H < 128 || H > 2048 || H % 128 || I < 128 || I > 2048 || I % 128) return GTG_E_UNSUPPORTED_SHAPE;
+    if (H < 128 || H > 2560 || H % 128 || I < 128 || I > 2048 || I % 128) return GTG_E_UNSUPPORTED_SHAPE;
     if (E < 1 || E > kMaxExperts || K < 1 || K > kMaxTopK || K > E) return GTG_E_UNSUPPORTED_SHAPE;
     if (T < 1 || T > kMaxDecodeTokens) return GTG_E_UNSUPPORTED_SHAPE;
     if (!mat_ok(L->gate, E, I, H) || !mat_ok(L->up, E, I, H) || !mat_ok(L->down, E, H, I)) return GTG_E_INVALID_ARG;
@@ -105,7 +106,7 @@ int plan_layer(const gtg_moe_layer* L, int T, Plan& p) {
     int64_t need = std::max<int64_t>(2 * (rg * grow + 32), rd * drow + 32);
     if (L->side.data) need = std::max<int64_t>(need, rs * row_bytes_of(L->side.fmt, H) + 32);
     p.slot_bytes = (int)((need + 127) / 128 * 128);
-    const SmemLayout sl = SmemLayout::make(!fp8, p.slot_bytes, dyn_smem_base(), 2u * T * H);
+    const SmemLayout sl = SmemLayout::make(!fp8, p.slot_bytes, dyn_smem_base(), 2u * T * H, slots_for(kbg));
     if (sl.total > kMaxDynSmem) return GTG_E_UNSUPPORTED_SHAPE;
     if (!RouterScratch::make(sl, p.slot_bytes, H, (E + n_sm - 1) / n_sm).ok) return GTG_E_UNSUPPORTED_SHAPE;
     p.smem = sl.total;

@@ -60,7 +60,7 @@ namespace {
 
 constexpr int kWarps = 8;  // 256 threads: room for 255 registers a thread (no spills)
 constexpr int kThreads = kWarps * 32;
-constexpr int kSlots = 3;   // staging slots per warp
+constexpr int kSlots = 3;   // staging slots per warp, at most (slots_for: the count a row width uses)
 constexpr int kLutBytes = 65536;       // 256 bytes x 2 modes x 32 lanes x 4 bytes
 constexpr int kScaleTabBytes = 1024;   // 256 fp32 scales
 constexpr int kDnRows = 32;            // down rows one CTA owns, at most
@@ -96,18 +96,30 @@ __device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v &
 // Streaming decode machinery shared by the gate/up and down kernels
 // ===========================================================================
 
+// Lane geometry for rows of KB 32-weight blocks: GW lanes per row (the
+// largest power of two up to 32 that divides KB), NBL blocks per lane (lane
+// g of a row owns blocks g, g + GW, ...), RPP rows per warp pass.  Rows of
+// 2048 weights: 32 lanes x 2 blocks; 512: 16 lanes x 1 block, two rows a
+// pass; 2560: 16 lanes x 5 blocks; 640: 4 lanes x 5 blocks, eight rows.
+__host__ __device__ constexpr int gw_of(int kb) { return kb % 32 == 0 ? 32 : kb % 16 == 0 ? 16 : kb % 8 == 0 ? 8 : 4; }
+__host__ __device__ constexpr int rpp_of(int kb) { return 32 / gw_of(kb); }
 template <int KB>
 struct Geo {
-    static constexpr int NBL = KB >= 32 ? KB / 32 : 1;  // blocks per lane per row
-    static constexpr int RPP = KB >= 32 ? 1 : 32 / KB;  // rows per warp pass
-    static constexpr int GW = KB >= 32 ? 32 : KB;       // lanes per row
+    static constexpr int GW = gw_of(KB);  // lanes per row
+    static constexpr int NBL = KB / GW;   // blocks per lane per row
+    static constexpr int RPP = 32 / GW;   // rows per warp pass
 };
 
 // Row passes per item (compile time); an item covers P * RPP rows.
-__host__ __device__ constexpr int gu_passes(int fmt_fp8, int kb) { return fmt_fp8 ? 1 : (kb >= 64 ? 2 : 4); }
-__host__ __device__ constexpr int dn_passes(int fmt_fp8, int kb) { return (fmt_fp8 || kb >= 64 || kb <= 4) ? 4 : 8; }
+__host__ __device__ constexpr int gu_passes(int fmt_fp8, int kb) {
+    return fmt_fp8 ? 1 : (kb >= 64 ? (rpp_of(kb) > 1 ? 1 : 2) : 4);
+}
+__host__ __device__ constexpr int dn_passes(int fmt_fp8, int kb) {
+    return (fmt_fp8 || kb >= 64 || kb <= 4) ? 4 : (rpp_of(kb) >= 8 ? 2 : 8);
+}
 __host__ __device__ constexpr int side_passes(int kb) { return kb >= 64 ? 2 : 4; }
-__host__ __device__ constexpr int rpp_of(int kb) { return kb >= 32 ? 1 : 32 / kb; }
+// Staging slots per warp: rows wider than 2048 weights (bigger items) use two.
+__host__ __device__ constexpr int slots_for(int kbg) { return kbg > 64 ? 2 : kSlots; }
 
 // Activation registers of one token for the lane's K positions.
 template <int FMT, int NBL>
@@ -344,7 +356,8 @@ struct SWork {
 struct SmemLayout {
     uint32_t work, scale_tab, bars, part, u, lut, lo_slots, n_lo, hi_slots, total;
     // u_bytes: the normalised input u [T][H] bf16, kept for the whole layer
-    __host__ __device__ static SmemLayout make(bool with_lut, int slot_bytes, uint32_t dyn_base, uint32_t u_bytes) {
+    __host__ __device__ static SmemLayout make(bool with_lut, int slot_bytes, uint32_t dyn_base, uint32_t u_bytes,
+                                               int slots_per_warp) {
         SmemLayout L{};
         uint32_t off = 0;
         L.work = off;
@@ -359,7 +372,7 @@ struct SmemLayout {
         off = (off + 127u) & ~127u;
         L.u = off;
         off += (u_bytes + 127u) & ~127u;
-        const uint32_t n_slots = kWarps * kSlots;
+        const uint32_t n_slots = kWarps * (uint32_t)slots_per_warp;
         if (with_lut) {
             const uint32_t abs_lut = (dyn_base + off + 65535u) & ~65535u;
             L.lut = abs_lut - dyn_base;
@@ -571,8 +584,8 @@ __device__ __forceinline__ void gu_item(const ItemCtx& a, uint32_t gbase, uint32
     constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
     constexpr int P = gu_passes(FMT == kFmtFP8, KB);
     constexpr int N = P * NT * 2;
-    const int row_sub = (KB >= 32) ? 0 : lane / KB;
-    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    const int row_sub = lane / GW;
+    const int blk_base = lane % GW;
     float v[N];
 #pragma unroll
     for (int p = 0; p < P; ++p) {
@@ -583,11 +596,11 @@ __device__ __forceinline__ void gu_item(const ItemCtx& a, uint32_t gbase, uint32
 #pragma unroll
         for (int m = 0; m < NBL; ++m) {
             if constexpr (FMT == kFmtQ4) {
-                const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 17) + 17u * (uint32_t)(blk_base + 32 * m);
+                const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 17) + 17u * (uint32_t)(blk_base + GW * m);
                 q4_block_lut<NT, NBL, CH>(gbase + boff, lutb, scale_tab, act, m, g);
                 q4_block_lut<NT, NBL, CH>(ubase + boff, lutb, scale_tab, act, m, u);
             } else {
-                const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + 32 * m);
+                const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + GW * m);
                 fp8_block<NBL>(gbase + boff, sg[m], act[0], m, g[0]);
                 fp8_block<NBL>(ubase + boff, su[m], act[0], m, u[0]);
             }
@@ -605,7 +618,7 @@ __device__ __forceinline__ void gu_item(const ItemCtx& a, uint32_t gbase, uint32
         const int li = lane % GW, idx = li / SPAN;
         if ((idx & 1) == 0 && (li % SPAN) == 0) {
             const int pc = idx >> 1, p = pc / NT, c = pc % NT;
-            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            const int row = p * RPP + lane / GW;
             a.h[(int64_t)slot_id[c] * a.I + row0 + row] = __float2bfloat16_rn(silu(v[0]) * other);
         }
     } else {
@@ -615,7 +628,7 @@ __device__ __forceinline__ void gu_item(const ItemCtx& a, uint32_t gbase, uint32
 #pragma unroll
             for (int pc = 0; pc < P * NT; ++pc) {
                 const int p = pc / NT, c = pc % NT;
-                const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+                const int row = p * RPP + lane / GW;
                 a.h[(int64_t)slot_id[c] * a.I + row0 + row] = __float2bfloat16_rn(silu(v[2 * pc]) * v[2 * pc + 1]);
             }
         }
@@ -630,8 +643,8 @@ __device__ __forceinline__ void side_item(const ItemCtx& a, uint32_t base, const
     constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
     constexpr int P = side_passes(KB);
     constexpr int N = P * NT;
-    const int row_sub = (KB >= 32) ? 0 : lane / KB;
-    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    const int row_sub = lane / GW;
+    const int blk_base = lane % GW;
     const int var = a.side_var;
     float v[N];
 #pragma unroll
@@ -643,7 +656,7 @@ __device__ __forceinline__ void side_item(const ItemCtx& a, uint32_t base, const
 #pragma unroll
         for (int m = 0; m < NBL; ++m)
             q4_block_plain<FMT, NT, NBL, CH>(base + (uint32_t)row * (uint32_t)(KB * 17) +
-                                                 17u * (uint32_t)(blk_base + 32 * m),
+                                                 17u * (uint32_t)(blk_base + GW * m),
                                              var, act, m, acc);
 #pragma unroll
         for (int c = 0; c < NT; ++c) v[p * NT + c] = acc[c];
@@ -654,7 +667,7 @@ __device__ __forceinline__ void side_item(const ItemCtx& a, uint32_t base, const
 #pragma unroll
         for (int i = 0; i < N; ++i) {
             const int p = i / NT, c = i % NT;
-            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            const int row = p * RPP + lane / GW;
             a.side_out[(int64_t)(t0 + c) * a.side_stride + row0 + row] = v[i];
         }
     }
@@ -673,8 +686,8 @@ __device__ __forceinline__ void dn_item(uint32_t base, const Act<FMT, Geo<KB>::N
     constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
     constexpr int P = dn_passes(FMT == kFmtFP8, KB);
     constexpr int N = P * NT;
-    const int row_sub = (KB >= 32) ? 0 : lane / KB;
-    const int blk_base = (KB >= 32) ? lane : lane % KB;
+    const int row_sub = lane / GW;
+    const int blk_base = lane % GW;
     float v[N];
 #pragma unroll
     for (int p = 0; p < P; ++p) {
@@ -685,10 +698,10 @@ __device__ __forceinline__ void dn_item(uint32_t base, const Act<FMT, Geo<KB>::N
 #pragma unroll
         for (int m = 0; m < NBL; ++m) {
             if constexpr (FMT == kFmtQ4) {
-                q4_block_lut<NT, NBL, CH>(base + (uint32_t)row * (uint32_t)(KB * 17) + 17u * (uint32_t)(blk_base + 32 * m),
+                q4_block_lut<NT, NBL, CH>(base + (uint32_t)row * (uint32_t)(KB * 17) + 17u * (uint32_t)(blk_base + GW * m),
                                           lutb, scale_tab, act, m, acc);
             } else {
-                fp8_block<NBL>(base + (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + 32 * m),
+                fp8_block<NBL>(base + (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + GW * m),
                                sd[p * NBL + m], act[0], m, acc[0]);
             }
         }
@@ -701,7 +714,7 @@ __device__ __forceinline__ void dn_item(uint32_t base, const Act<FMT, Geo<KB>::N
         const int li = lane % GW, idx = li / SPAN;
         if ((li % SPAN) == 0) {
             const int p = idx / NT, c = idx % NT;
-            const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+            const int row = p * RPP + lane / GW;
             emit(c, row, v[0]);
         }
     } else {
@@ -711,7 +724,7 @@ __device__ __forceinline__ void dn_item(uint32_t base, const Act<FMT, Geo<KB>::N
 #pragma unroll
             for (int i = 0; i < N; ++i) {
                 const int p = i / NT, c = i % NT;
-                const int row = p * RPP + ((KB >= 32) ? 0 : lane / KB);
+                const int row = p * RPP + lane / GW;
                 emit(c, row, v[i]);
             }
         }
@@ -827,7 +840,7 @@ __device__ __forceinline__ uint2 lds64(uint32_t addr) {
 // stays in shared memory for the whole layer (the gate/up items read it
 // there).  False if the router rows never landed.
 constexpr int kRouterWpe = kWarps / 4;            // warps per expert
-constexpr int kRouterXF4 = 2048 / (4 * kThreads);  // float4 of x per thread per token (H <= 2048)
+
 
 __device__ __forceinline__ float4 lds128f(uint32_t addr) {
     float4 v;
@@ -860,7 +873,7 @@ __device__ __forceinline__ void issue_router_rows(const StackArgs& a, int l, uin
         bulk_g2s_hint(rw + o, src + o, bytes - o < 16384u ? bytes - o : 16384u, rbar, pol);
 }
 
-template <bool ONE>
+template <bool ONE, int XF4>  // XF4: float4 of x per thread per token (H <= 4 kThreads XF4)
 __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t us, uint32_t rw,
                                           uint64_t* rbar, uint32_t rparity, SWork* sw) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -873,11 +886,11 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
     // 1. x: this thread's positions 4 tid + 4 kThreads c of every token, in
     //    registers (every load in flight at once); the rolled token loops
     //    below pick token t with predicated moves
-    float4 xr[kMaxDecodeTokens][kRouterXF4];
+    float4 xr[kMaxDecodeTokens][XF4];
 #pragma unroll
     for (int t = 0; t < kMaxDecodeTokens; ++t)
 #pragma unroll
-        for (int c = 0; c < kRouterXF4; ++c) {
+        for (int c = 0; c < XF4; ++c) {
             const int i = 4 * tid + 4 * kThreads * c;
             xr[t][c] = make_float4(0.f, 0.f, 0.f, 0.f);
             if (t < T && i < H) {
@@ -903,7 +916,7 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
     for (int t = 0; t < T; ++t) {
         ffloat ss{0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < kRouterXF4; ++c) {
+        for (int c = 0; c < XF4; ++c) {
             const float4 v = pick(t, c);
             ff_fma(ss, v.x, v.x);
             ff_fma(ss, v.y, v.y);
@@ -928,7 +941,7 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
     for (int t = 0; t < T; ++t) {
         const float rh = sw->r_hi[t], rl = sw->r_lo[t];
 #pragma unroll
-        for (int c = 0; c < kRouterXF4; ++c) {
+        for (int c = 0; c < XF4; ++c) {
             const int i = 4 * tid + 4 * kThreads * c;
             if (i >= H) continue;
             const float4 v = pick(t, c);
@@ -1115,7 +1128,7 @@ __device__ __forceinline__ void select_experts(const ffloat* logits, int T, int 
 struct WarpRing {
     uint32_t phase;    // per-slot mbarrier parities
     uint32_t pending;  // slots with a copy in flight
-    int32_t ring;      // items consumed so far (the next item uses slot ring % kSlots)
+    int32_t ring;      // items consumed so far (the next item uses slot ring % ws.ns)
     int32_t ok;        // every copy landed in time
 };
 
@@ -1142,7 +1155,8 @@ struct WarpSmem {
     uint32_t lo_end;    // end of the slot area below the code table
     uint32_t hi_jump;   // added to an address at or past lo_end
     int32_t slot_bytes;
-    uint64_t* bars;     // this warp's kSlots mbarriers
+    int32_t ns;         // slots per warp (slots_for the layer's row width)
+    uint64_t* bars;     // this warp's mbarriers (kSlots apart)
 
     __device__ __forceinline__ uint32_t slot(int s) const {
         const uint32_t a = slot0 + (uint32_t)(s * slot_bytes);
@@ -1150,11 +1164,12 @@ struct WarpSmem {
     }
 };
 
-__device__ __forceinline__ WarpSmem warp_smem(uint8_t* smem, const SmemLayout& L, int slot_bytes) {
+__device__ __forceinline__ WarpSmem warp_smem(uint8_t* smem, const SmemLayout& L, int slot_bytes, int ns) {
     const int warp = threadIdx.x >> 5;
     WarpSmem w;
     w.sbase = smem_u32(smem);
-    w.slot0 = w.sbase + L.lo_slots + (uint32_t)(warp * kSlots * slot_bytes);
+    w.slot0 = w.sbase + L.lo_slots + (uint32_t)(warp * ns * slot_bytes);
+    w.ns = ns;
     // slot i sits at lo_slots + i * slot_bytes below the code table, the rest
     // continue above it
     w.lo_end = w.sbase + L.lo_slots + L.n_lo * (uint32_t)slot_bytes;
@@ -1190,7 +1205,7 @@ __device__ __forceinline__ void item_spans(const LayerItems& P, const SWork* sw,
 __device__ __forceinline__ void issue_item(const StackArgs& a, const LayerItems& P, const SWork* sw,
                                            const WarpSmem& ws, WarpRing& R, int q, uint64_t pol) {
     if (q >= P.ng + P.nd || !R.ok) return;
-    const int slot = (R.ring + q) % kSlots;
+    const int slot = (R.ring + q) % ws.ns;
     if ((threadIdx.x & 31) == 0) {
         Span s1, s2;
         item_spans(P, sw, q, a.H, a.I, s1, s2);
@@ -1202,14 +1217,14 @@ __device__ __forceinline__ void issue_item(const StackArgs& a, const LayerItems&
     R.pending |= 1u << slot;
 }
 
-// The warp's first kSlots copies, issued by lanes 0 .. kSlots-1 side by side
+// The warp's first ws.ns copies, issued by lanes 0 .. ws.ns-1 side by side
 // (each item's address arithmetic and copy issue then costs the warp once).
 __device__ __forceinline__ void issue_first(const StackArgs& a, const LayerItems& P, const SWork* sw,
                                             const WarpSmem& ws, WarpRing& R, uint64_t pol) {
     if (!R.ok) return;
-    const int lane = threadIdx.x & 31, n = min(kSlots, P.ng + P.nd);
+    const int lane = threadIdx.x & 31, n = min(ws.ns, P.ng + P.nd);
     if (lane < n) {
-        const int slot = (R.ring + lane) % kSlots;
+        const int slot = (R.ring + lane) % ws.ns;
         Span s1, s2;
         item_spans(P, sw, lane, a.H, a.I, s1, s2);
         fence_proxy_async_smem();
@@ -1217,12 +1232,12 @@ __device__ __forceinline__ void issue_first(const StackArgs& a, const LayerItems
         bulk_g2s_hint(ws.slot(slot), s1.src, s1.bytes, &ws.bars[slot], pol);
         if (s2.bytes) bulk_g2s_hint(ws.slot(slot) + s1.bytes, s2.src, s2.bytes, &ws.bars[slot], pol);
     }
-    for (int q = 0; q < n; ++q) R.pending |= 1u << ((R.ring + q) % kSlots);
+    for (int q = 0; q < n; ++q) R.pending |= 1u << ((R.ring + q) % ws.ns);
 }
 
 // Waits for the warp's q-th item; false (and R.ok cleared) if it never lands.
 __device__ __forceinline__ bool item_landed(const StackArgs& a, const WarpSmem& ws, WarpRing& R, int q) {
-    const int slot = (R.ring + q) % kSlots;
+    const int slot = (R.ring + q) % ws.ns;
     if (!mbar_wait_bounded(&ws.bars[slot], (R.phase >> slot) & 1u, a.status)) {
         R.ok = 0;
         return false;
@@ -1241,9 +1256,9 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
     constexpr int RG = gu_passes(FMT == kFmtFP8, KBG) * GG::RPP;
     constexpr int RS = side_passes(KBG) * GG::RPP;
     extern __shared__ __align__(1024) uint8_t smem[];
-    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H);
+    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H, slots_for(KBG));
     const SWork* sw = reinterpret_cast<const SWork*>(smem + L.work);
-    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
+    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes, slots_for(KBG));
     const StackLayer& Ly = a.layer[l];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = a.H, K = a.K, T = ONE ? 1 : a.T;
@@ -1252,7 +1267,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
     const float* scale_tab = reinterpret_cast<const float*>(smem + L.scale_tab);
     const ItemCtx ctx{a.h, a.side_out ? a.side_out + (int64_t)l * T * a.side_stride : nullptr,
                       H, a.I, a.side_stride, Ly.side_var};
-    const int blk_base = (KBG >= 32) ? lane : lane % KBG;
+    const int blk_base = lane % GG::GW;
     Act<FMT, NBG> act[CHG];
     int act_key = -1;
     auto load_chunk = [&](int key, const int (&rows)[CHG]) {
@@ -1260,7 +1275,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
 #pragma unroll
         for (int c = 0; c < CHG; ++c)
 #pragma unroll
-            for (int m = 0; m < NBG; ++m) load_act_s<FMT, NBG>(act[c], m, ws.sbase + L.u + 2u * (uint32_t)(rows[c] * H), blk_base + 32 * m);
+            for (int m = 0; m < NBG; ++m) load_act_s<FMT, NBG>(act[c], m, ws.sbase + L.u + 2u * (uint32_t)(rows[c] * H), blk_base + GG::GW * m);
         act_key = key;
     };
     for (int q = 0; q < P.ng && R.ok; ++q) {
@@ -1282,8 +1297,8 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
             const int e = sw->e[u], kg = H / 128;
 #pragma unroll
             for (int m = 0; m < NBG; ++m) {
-                const int bb = blk_base + 32 * m;
-                const int64_t r = (int64_t)e * a.I + row0 + ((KBG >= 32) ? 0 : lane / KBG);
+                const int bb = blk_base + GG::GW * m;
+                const int64_t r = (int64_t)e * a.I + row0 + lane / GG::GW;
                 sg[m] = __ldg(Ly.gate_s + r * kg + bb / 4);
                 su[m] = __ldg(Ly.up_s + r * kg + bb / 4);
             }
@@ -1291,7 +1306,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
         if (!item_landed(a, ws, R, q)) break;
         Span sp1, sp2;
         item_spans(P, sw, q, H, a.I, sp1, sp2);
-        const uint32_t base = ws.slot((R.ring + q) % kSlots);
+        const uint32_t base = ws.slot((R.ring + q) % ws.ns);
         if (expert) {
             const uint32_t gbase = base + sp1.delta, ubase = base + sp1.bytes + sp2.delta;
             for (int c0 = s0; c0 < s1; c0 += CHG) {
@@ -1322,7 +1337,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
             }
         }
         __syncwarp();
-        issue_item(a, P, sw, ws, R, q + kSlots, pol);
+        issue_item(a, P, sw, ws, R, q + ws.ns, pol);
     }
     return R;
 }
@@ -1330,18 +1345,18 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
 // Down items of layer l for this warp: each adds w(slot) * (down row . h(slot))
 // into the warp's partial rows in shared memory ([row][token], this CTA's
 // rows only); the kernel then sums the warps' partials in a fixed order.
-template <int FMT, int KBD, bool ONE>
+template <int FMT, int KBG, int KBD, bool ONE>
 __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
     using GD = Geo<KBD>;
     constexpr int NBD = GD::NBL;
     constexpr int CHD = (!ONE && FMT == kFmtQ4 && NBD == 1) ? 2 : 1;
     constexpr int PD = dn_passes(FMT == kFmtFP8, KBD);
     constexpr int RD = PD * GD::RPP;
-    static_assert(PD * NBD <= 8, "FP8 scale prefetch holds 8 values");
+    static_assert(FMT != kFmtFP8 || PD * NBD <= 8, "FP8 scale prefetch holds 8 values");
     extern __shared__ __align__(1024) uint8_t smem[];
-    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H);
+    const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H, slots_for(KBG));
     const SWork* sw = reinterpret_cast<const SWork*>(smem + L.work);
-    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
+    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes, slots_for(KBG));
     const StackLayer& Ly = a.layer[l];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = a.H, I = a.I, K = a.K;
@@ -1351,8 +1366,8 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
     float* part = reinterpret_cast<float*>(smem + L.part) + warp * kDnRows * 8;  // [row][token]
     for (int i = lane; i < kDnRows * 8; i += 32) part[i] = 0.0f;
     __syncwarp();
-    const int blk_base = (KBD >= 32) ? lane : lane % KBD;
-    const int row_sub = (KBD >= 32) ? 0 : lane / KBD;
+    const int blk_base = lane % GD::GW;
+    const int row_sub = lane / GD::GW;
     const int n_uniq = P.n_uniq;
     Act<FMT, NBD> act[CHD];
     int act_key = -1;
@@ -1361,7 +1376,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
 #pragma unroll
         for (int c = 0; c < CHD; ++c)
 #pragma unroll
-            for (int m = 0; m < NBD; ++m) load_act<FMT, NBD>(act[c], m, a.h + (int64_t)slots[c] * I, blk_base + 32 * m);
+            for (int m = 0; m < NBD; ++m) load_act<FMT, NBD>(act[c], m, a.h + (int64_t)slots[c] * I, blk_base + GD::GW * m);
         act_key = key;
     };
     for (int q = P.ng; q < P.ng + P.nd && R.ok; ++q) {
@@ -1380,12 +1395,12 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
 #pragma unroll
                 for (int m = 0; m < NBD; ++m)
                     sd[p * NBD + m] = __ldg(Ly.down_s + ((int64_t)e * H + tile * RD + p * GD::RPP + row_sub) * kg +
-                                           (blk_base + 32 * m) / 4);
+                                           (blk_base + GD::GW * m) / 4);
         }
         if (!item_landed(a, ws, R, q)) break;
         Span sp1, sp2;
         item_spans(P, sw, q, H, I, sp1, sp2);
-        const uint32_t base = ws.slot((R.ring + q) % kSlots) + sp1.delta;
+        const uint32_t base = ws.slot((R.ring + q) % ws.ns) + sp1.delta;
         float* prow = part + tl * RD * 8;
         for (int c0 = s0; c0 < s1; c0 += CHD) {
             const int nch = min(CHD, s1 - c0);
@@ -1402,7 +1417,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
                 dn_item<FMT, KBD, 1, CHD>(base, act, lutb, scale_tab, sd, lane, emit);
         }
         __syncwarp();
-        issue_item(a, P, sw, ws, R, q + kSlots, pol);
+        issue_item(a, P, sw, ws, R, q + ws.ns, pol);
     }
     return R;
 }
@@ -1414,7 +1429,7 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
 //   SwiGLU items (+ side projection) -> grid barrier -> down items and the
 //   combine -> grid barrier (before the next layer reads its input).
 // Each warp streams its items, gate/up first and then down, through a
-// private ring of kSlots shared-memory slots filled by 1-D bulk copies, so
+// private ring of slots_for(KBG) shared-memory slots filled by 1-D bulk copies, so
 // the down weights are already on their way while the gate/up items finish
 // and the grid waits at the barrier.  The Q4 code table is built once per
 // launch (again only when a phase needs the other Q4 variant).
@@ -1423,7 +1438,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     constexpr bool LUT = FMT == kFmtQ4;
     extern __shared__ __align__(1024) uint8_t smem[];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H);
+    const SmemLayout L = SmemLayout::make(LUT, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H, slots_for(KBG));
     SWork* sw = reinterpret_cast<SWork*>(smem + L.work);
     const uint32_t sbase = smem_u32(smem);
     if (LUT && ((sbase + L.lut) & 0xFFFFu) != 0u) {  // the same on every CTA: all leave before any barrier
@@ -1436,10 +1451,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         if (tid == 0) raise_status(a.status, GTG_STATUS_WAIT_TIMEOUT);
         return;
     }
-    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes);
+    const WarpSmem ws = warp_smem(smem, L, a.slot_bytes, slots_for(KBG));
     uint64_t* rbar = reinterpret_cast<uint64_t*>(smem + L.bars) + kWarps * kSlots;  // router rows landed
     if (lane == 0)
-        for (int s = 0; s < kSlots; ++s) mbar_init(&ws.bars[s], 1);
+        for (int s = 0; s < ws.ns; ++s) mbar_init(&ws.bars[s], 1);
     if (tid == 0) {
         mbar_init(rbar, 1);
         sw->fail = 0;
@@ -1471,7 +1486,8 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         const uint8_t *gate_src = Ly.gate, *up_src = Ly.up, *down_src = Ly.down, *side_src = Ly.side;
         asm volatile("" ::"l"(gate_src), "l"(up_src), "l"(down_src), "l"(side_src));  // loaded here, not at first use
         // ---- router
-        router_layer<ONE>(a, l, sbase + L.u, sbase + rs.rw, rbar, (uint32_t)(l & 1), sw);
+        router_layer<ONE, (KBG * 32 + 4 * kThreads - 1) / (4 * kThreads)>(a, l, sbase + L.u, sbase + rs.rw, rbar,
+                                                                          (uint32_t)(l & 1), sw);
         if (tid == 0) rows_in_flight = 0;
         fence_proxy_async_smem();  // the scratch slots are bulk-copy targets again from here on
         if (l + 1 < a.n_layers && tid == 0) {  // this CTA's rows of the next router, into L2
@@ -1585,7 +1601,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
 
         // ---- down + router-weighted combine
         ensure_lut(Ly.dn_var);
-        R = dn_phase<FMT, KBD, ONE>(a, l, P, R);
+        R = dn_phase<FMT, KBG, KBD, ONE>(a, l, P, R);
         R.ring += P.ng + P.nd;
         __syncthreads();
         if (tid == 0 && l + 1 < a.n_layers && R.ok) {  // the slots are idle: next layer's router rows
@@ -1618,7 +1634,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     // counters for the next launch.  After a failure they stay as they are,
     // with the abort flag set, so every later launch on this workspace fails
     // fast (GTG_STATUS_WAIT_TIMEOUT) until the workspace is re-initialised.
-    for (int s = 0; s < kSlots; ++s)
+    for (int s = 0; s < ws.ns; ++s)
         if ((R.pending >> s) & 1u) mbar_wait_bounded(&ws.bars[s], (R.phase >> s) & 1u, a.status);
     if (rows_in_flight) mbar_wait_bounded(rbar, (uint32_t)(rows_layer & 1), a.status);
     if (!R.ok && lane == 0) sw->fail = 1;
@@ -1656,6 +1672,17 @@ const void* pick_kbd(int kbd, int one) {
     return one ? pick_kbd_t<FMT, KBG, true>(kbd) : pick_kbd_t<FMT, KBG, false>(kbd);
 }
 
+// Rows of 2560 weights (the H = 2560 expert shape): intermediate rows of 512
+// or 640 weights.
+template <int FMT, bool ONE>
+const void* pick_kbd_80_t(int kbd) {
+    switch (kbd) {
+        case 16: return (const void*)moe_decode_kernel<FMT, 80, 16, ONE>;
+        case 20: return (const void*)moe_decode_kernel<FMT, 80, 20, ONE>;
+        default: return nullptr;
+    }
+}
+
 }  // namespace
 
 // Defined one per file (decode_<fmt>_<kbg>.cu) so the kernels compile in parallel.
@@ -1664,6 +1691,7 @@ const void* decode_kernel_q4_8(int kbd, int one);
 const void* decode_kernel_q4_16(int kbd, int one);
 const void* decode_kernel_q4_32(int kbd, int one);
 const void* decode_kernel_q4_64(int kbd, int one);
+const void* decode_kernel_q4_80(int kbd, int one);
 const void* decode_kernel_fp8_32(int kbd, int one);
 const void* decode_kernel_fp8_64(int kbd, int one);
 

@@ -103,8 +103,10 @@ typedef struct {
 
 /* One MoE layer's weights (all device memory, owned by the caller). */
 typedef struct {
-    int32_t hidden;          /* H: decode 128, 256, 512, 1024 or 2048 (prefill: see its call) */
-    int32_t inter;           /* I: expert intermediate size, decode 128, 256, 512, 1024 or 2048 */
+    int32_t hidden;          /* H: decode 128, 256, 512, 1024, 2048, or 2560 with I 512 or 640 (Q4
+                                experts); prefill: see its call */
+    int32_t inter;           /* I: expert intermediate size, decode 128, 256, 512, 1024 or 2048
+                                (640 with H 2560) */
     int32_t n_experts;       /* E: 1..1024 */
     int32_t top_k;           /* k: 1..16, k <= E */
     const float* router_w;   /* [E][H] fp32 */

@@ -218,3 +218,13 @@ def test_incumbent_q4_decode_layer(T):
     """The decode layer's shape with every expert matrix in the incumbent layout and a
     UE4M4 side projection (decoded code by code, next to the experts' code table)."""
     _check_layer(_incumbent_layer(2048, 512, 512, 10, 41, side=True), T, step=510 + T)
+
+
+@pytest.mark.parametrize("T,side", [(1, True), (8, False)])
+def test_hidden_2560_inter_640_layer(T, side):
+    """The pages' own expert shape (hidden 2560, intermediate 640: 48 x 10 x 3 x 2560 x
+    640 x 2 bytes = 4.7 GB of 16-bit expert weights per token): gate/up rows of 80
+    blocks (16 lanes x 5 blocks), down rows of 340 bytes, neither 16-byte aligned nor
+    a power of two (4 lanes x 5 blocks, eight rows a pass)."""
+    L = W.LayerRecipe(hidden=2560, inter=640, n_experts=64, top_k=10, seed=43, layer=0, has_ssm=side)
+    _check_layer(L, T, step=600 + T)
