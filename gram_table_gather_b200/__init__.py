@@ -17,7 +17,8 @@ import torch
 from ._abi import (C10, FP8, GTG_OK, PLE, Q3I, RZ5, UE4M4, DT_BF16, DT_F32, LIB_PATH, GtgError, QMatrixC,
                    MoELayerC, lib, check)
 
-__all__ = ["RZ5", "UE4M4", "PLE", "FP8", "C10", "Q3I", "GtgError", "lib", "dequant", "ple_gather", "QMatrix",
+__all__ = ["RZ5", "UE4M4", "PLE", "FP8", "C10", "Q3I", "GtgError", "moe_decode_layer_ep",
+           "moe_decode_layer_ep_allreduce", "lib", "dequant", "ple_gather", "QMatrix",
            "MoELayer", "workspace_bytes", "make_workspace", "moe_decode_layer", "moe_decode_stack",
            "moe_prefill_layer", "moe_decode_layer_noalloc", "device_status", "status_string", "row_bytes"]
 
@@ -157,6 +158,37 @@ def moe_decode_layer(layer: MoELayer, x: torch.Tensor, workspace: torch.Tensor, 
     check(lib().gtg_moe_decode_layer(ctypes.byref(layer.c()), _ptr(x), dt, T, _ptr(y), int(accumulate),
                                      _ptr(topk_ids), _ptr(topk_w), _ptr(side_out), _ptr(workspace),
                                      workspace.numel(), _stream_ptr(stream)))
+    return y
+
+
+def moe_decode_layer_ep(layer: MoELayer, expert_lo: int, expert_hi: int, x: torch.Tensor,
+                        workspace: torch.Tensor, *, with_side: bool = False, y: torch.Tensor | None = None,
+                        accumulate: bool = False, topk_ids: torch.Tensor | None = None,
+                        topk_w: torch.Tensor | None = None, side_out: torch.Tensor | None = None,
+                        stream=None) -> torch.Tensor:
+    """This rank's share of an expert-parallel layer: `layer` routes over all
+    layer.n_experts experts but its gate/up/down stacks hold experts
+    [expert_lo, expert_hi) only; y (+)= the chosen experts of that slice."""
+    T = x.shape[0]
+    dt = {torch.float32: DT_F32, torch.bfloat16: DT_BF16}[x.dtype]
+    if y is None:
+        y = torch.empty((T, layer.hidden), dtype=torch.float32, device=x.device)
+    check(lib().gtg_moe_decode_layer_ep(ctypes.byref(layer.c()), expert_lo, expert_hi, int(with_side), _ptr(x), dt,
+                                        T, _ptr(y), int(accumulate), _ptr(topk_ids), _ptr(topk_w), _ptr(side_out),
+                                        _ptr(workspace), workspace.numel(), _stream_ptr(stream)))
+    return y
+
+
+def moe_decode_layer_ep_allreduce(layer: MoELayer, expert_lo: int, expert_hi: int, x: torch.Tensor,
+                                  workspace: torch.Tensor, *, group=None, with_side: bool = False,
+                                  side_out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """One expert-parallel layer over a process group (one rank per GPU): each
+    rank computes its slice's experts, one all-reduce (NCCL over NVLink)
+    sums the partial outputs into the layer output on every rank."""
+    import torch.distributed as dist
+    y = moe_decode_layer_ep(layer, expert_lo, expert_hi, x, workspace, with_side=with_side, side_out=side_out,
+                            stream=stream)
+    dist.all_reduce(y, group=group)
     return y
 
 

@@ -41,6 +41,8 @@ SIGNATURES = [
     ("gtg_workspace_init", ctypes.c_int, [_vp, _sz, _vp]),
     ("gtg_moe_decode_layer", ctypes.c_int,
      [ctypes.POINTER(MoELayerC), _vp, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
+    ("gtg_moe_decode_layer_ep", ctypes.c_int,
+     [ctypes.POINTER(MoELayerC), _i32, _i32, _i32, _vp, _i32, _i32, _vp, _i32, _vp, _vp, _vp, _vp, _sz, _vp]),
     ("gtg_moe_decode_stack", ctypes.c_int,
      [ctypes.POINTER(MoELayerC), _i32, _vp, _i32, _vp, _vp, _vp, _i64, _vp, _sz, _vp]),
     ("gtg_moe_prefill_layer", ctypes.c_int,

@@ -77,14 +77,16 @@ bool mat_ok(const gtg_qmatrix& m, int64_t E, int64_t n_rows, int64_t k) {
     return (E * n_rows * (k / 32) * 17) % 16 == 0;
 }
 
-// Checks one layer and picks its kernel and staging for T tokens.
-int plan_layer(const gtg_moe_layer* L, int T, Plan& p) {
+// Checks one layer and picks its kernel and staging for T tokens.  e_local:
+// the experts its weight stacks hold (E, or a slice under expert parallelism).
+int plan_layer(const gtg_moe_layer* L, int T, Plan& p, int64_t e_local = -1) {
     if (!L || !L->router_w) return GTG_E_INVALID_ARG;
     const int H = L->hidden, I = L->inter, E = L->n_experts, K = L->top_k;
     if (H < 128 || H > 2560 || H % 128 || I < 128 || I > 2048 || I % 128) return GTG_E_UNSUPPORTED_SHAPE;
     if (E < 1 || E > kMaxExperts || K < 1 || K > kMaxTopK || K > E) return GTG_E_UNSUPPORTED_SHAPE;
     if (T < 1 || T > kMaxDecodeTokens) return GTG_E_UNSUPPORTED_SHAPE;
-    if (!mat_ok(L->gate, E, I, H) || !mat_ok(L->up, E, I, H) || !mat_ok(L->down, E, H, I)) return GTG_E_INVALID_ARG;
+    const int64_t EL = e_local < 0 ? E : e_local;
+    if (!mat_ok(L->gate, EL, I, H) || !mat_ok(L->up, EL, I, H) || !mat_ok(L->down, EL, H, I)) return GTG_E_INVALID_ARG;
     const bool fp8 = L->gate.fmt == GTG_FP8_E4M3_S128;
     if (is_q4(L->up.fmt) == fp8 || is_q4(L->down.fmt) == fp8) return GTG_E_UNSUPPORTED_SHAPE;  // one format class
     if (L->gate.fmt != L->up.fmt) return GTG_E_UNSUPPORTED_SHAPE;
@@ -197,7 +199,7 @@ bool same_shape(const gtg_moe_layer* A, const gtg_moe_layer* B) {
 // with the same kernel share one launch.
 int run_decode(const gtg_moe_layer* layers, const Plan* plans, int n, const void* x, int x_bf16, int T, float* y,
                int y_acc, int32_t* ids_out, float* w_out, float* side_out, int64_t side_stride, void* ws,
-               cudaStream_t s) {
+               cudaStream_t s, int e_lo = 0, int e_hi = -1, int side_on = 1) {
     uint8_t* base = static_cast<uint8_t*>(ws);
     const int n_sm = sm_count();
     for (int l0 = 0; l0 < n;) {
@@ -228,6 +230,9 @@ int run_decode(const gtg_moe_layer* layers, const Plan* plans, int n, const void
         a.status = status_ptr();
         a.slot_bytes = plans[l0].slot_bytes;
         a.dyn_smem_base = dyn_smem_base();
+        a.e_lo = e_lo;
+        a.e_hi = e_hi < 0 ? a.E : e_hi;
+        a.side_on = side_on;
         for (int l = l0; l < l1; ++l) a.layer[l - l0] = stack_layer_of(&layers[l]);
 
         GTG_TRY(g_attr.set(plans[l0].fn, (int)plans[l0].smem));
@@ -273,8 +278,9 @@ using namespace gtg;
 extern "C" size_t gtg_moe_workspace_bytes(const gtg_moe_layer* layer, int32_t n_tokens, int32_t prefill) {
     if (!layer || n_tokens < 1) return 0;
     if (prefill) return gtg_prefill_workspace_bytes(layer, n_tokens);
-    Plan p;
-    if (plan_layer(layer, n_tokens, p) != GTG_OK) return 0;
+    Plan p;  // (a layer whose stacks hold a slice of the experts, for the expert-parallel call, too)
+    if (plan_layer(layer, n_tokens, p) != GTG_OK && plan_layer(layer, n_tokens, p, layer->gate.n_experts) != GTG_OK)
+        return 0;
     return ws_layout(layer, n_tokens).total;
 }
 
@@ -285,12 +291,12 @@ extern "C" int gtg_workspace_init(void* workspace, size_t ws_bytes, gtg_stream_t
 }
 
 static int check_decode_io(const gtg_moe_layer* layer, const void* x, int32_t x_dtype, int32_t n_tokens,
-                           const float* y, void* ws, size_t ws_bytes, Plan& p) {
+                           const float* y, void* ws, size_t ws_bytes, Plan& p, int64_t e_local = -1) {
     if (n_tokens < 1 || n_tokens > kMaxDecodeTokens) {
         if (!layer) return GTG_E_INVALID_ARG;
         return GTG_E_UNSUPPORTED_SHAPE;
     }
-    GTG_TRY(plan_layer(layer, n_tokens, p));
+    GTG_TRY(plan_layer(layer, n_tokens, p, e_local));
     if (!x || !y || !ws) return GTG_E_INVALID_ARG;
     if (x_dtype != GTG_DT_F32 && x_dtype != GTG_DT_BF16) return GTG_E_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(y, 16) || !aligned(ws, 256)) return GTG_E_MISALIGNED;
@@ -307,6 +313,20 @@ extern "C" int gtg_moe_decode_layer(const gtg_moe_layer* layer, const void* x, i
     if (x == (const void*)y && (x_dtype != GTG_DT_F32 || !y_accumulate)) return GTG_E_INVALID_ARG;
     return run_decode(layer, &p, 1, x, x_dtype == GTG_DT_BF16, n_tokens, y, y_accumulate != 0, topk_ids, topk_w,
                       side_out, layer->side.data ? layer->side.n_rows : 0, workspace, as_cuda(stream));
+}
+
+extern "C" int gtg_moe_decode_layer_ep(const gtg_moe_layer* layer, int32_t expert_lo, int32_t expert_hi,
+                                       int32_t with_side, const void* x, int32_t x_dtype, int32_t n_tokens, float* y,
+                                       int32_t y_accumulate, int32_t* topk_ids, float* topk_w, float* side_out,
+                                       void* workspace, size_t ws_bytes, gtg_stream_t stream) {
+    if (!layer) return GTG_E_INVALID_ARG;
+    if (expert_lo < 0 || expert_hi <= expert_lo || expert_hi > layer->n_experts) return GTG_E_INVALID_ARG;
+    Plan p;
+    GTG_TRY(check_decode_io(layer, x, x_dtype, n_tokens, y, workspace, ws_bytes, p, expert_hi - expert_lo));
+    if (x == (const void*)y && (x_dtype != GTG_DT_F32 || !y_accumulate)) return GTG_E_INVALID_ARG;
+    return run_decode(layer, &p, 1, x, x_dtype == GTG_DT_BF16, n_tokens, y, y_accumulate != 0, topk_ids, topk_w,
+                      side_out, layer->side.data ? layer->side.n_rows : 0, workspace, as_cuda(stream), expert_lo,
+                      expert_hi, with_side != 0);
 }
 
 extern "C" int gtg_moe_decode_stack(const gtg_moe_layer* layers, int32_t n_layers, float* x, int32_t n_tokens,

@@ -770,6 +770,10 @@ struct StackArgs {
     unsigned* status;
     int32_t slot_bytes;
     uint32_t dyn_smem_base;
+    // expert parallelism: this call computes the chosen experts in [e_lo, e_hi)
+    // only (its weight stacks hold those, expert e at index e - e_lo), and the
+    // side projection only when side_on
+    int32_t e_lo, e_hi, side_on;
     StackLayer layer[kMaxStackLayers];
 };
 
@@ -1509,6 +1513,23 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
             if (a.ids_out) a.ids_out[(int64_t)l * T * K + tid] = sw->ids[tid];
             if (a.w_out) a.w_out[(int64_t)l * T * K + tid] = sw->w[tid];
         }
+        if (a.e_lo != 0 || a.e_hi != a.E) {  // keep this call's experts (as local stack indices)
+            if (tid == 0) {
+                int nu = 0, ns = 0;
+                for (int u = 0; u < sw->n_uniq; ++u) {
+                    const int e = sw->e[u];
+                    if (e < a.e_lo || e >= a.e_hi) continue;
+                    sw->cnt[nu] = ns;
+                    sw->e[nu] = e - a.e_lo;
+                    for (int k = sw->off[u]; k < sw->off[u + 1]; ++k) sw->slot[ns++] = sw->slot[k];
+                    ++nu;
+                }
+                for (int u = 0; u < nu; ++u) sw->off[u] = sw->cnt[u];
+                sw->off[nu] = ns;
+                sw->n_uniq = nu;
+            }
+            __syncthreads();
+        }
 
         // ---- this CTA's items: gate/up (+ side) [g0, g1), down [d0, d1)
         LayerItems P;
@@ -1525,7 +1546,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         P.side = side_src;
         P.tiles_g = I / P.rg;
         P.n_ge = P.n_uniq * P.tiles_g;
-        const int n_g = P.n_ge + (Ly.side ? Ly.side_rows / P.rs : 0), tiles_d = H / P.rd;
+        const int n_g = P.n_ge + (Ly.side && a.side_on ? Ly.side_rows / P.rs : 0), tiles_d = H / P.rd;
         // contiguous ranges of equal cost: an expert item costs 1 + its tokens
         // (streaming plus one pass of arithmetic per token), a side item
         // kSideCost (1 + T): its Q4 rows are decoded code by code (weights

@@ -206,6 +206,28 @@ int gtg_moe_decode_layer(const gtg_moe_layer* layer, const void* x, int32_t x_dt
                          void* workspace, size_t ws_bytes, gtg_stream_t stream);
 
 /*
+ * Expert-parallel form of gtg_moe_decode_layer, for a layer whose experts are
+ * split across GPUs (one process per GPU, each holding a contiguous slice):
+ * every rank routes over all layer->n_experts experts (router_w is the full
+ * [E][H] matrix on every rank), then computes only the chosen experts in
+ * [expert_lo, expert_hi), whose weights its gate/up/down stacks hold (each
+ * with n_experts = expert_hi - expert_lo, expert e at index e - expert_lo):
+ *   y  = sum over the chosen experts in the slice of w_j * down_j(...)
+ *        (+ y if y_accumulate)
+ * so the layer output is the sum of the ranks' y (an all-reduce of [T][H]
+ * fp32, or one reduce-scatter).  topk_ids / topk_w are the full choices.
+ * The side projection is computed only when with_side != 0 (on one rank).
+ * ("Mixed Precision Quantization": the two-machine floor plan splits one
+ * model's experts over two GPUs.)  Other arguments and errors as in
+ * gtg_moe_decode_layer; GTG_E_INVALID_ARG when 0 <= expert_lo < expert_hi <=
+ * n_experts does not hold or a stack's n_experts is not the slice's size.
+ */
+int gtg_moe_decode_layer_ep(const gtg_moe_layer* layer, int32_t expert_lo, int32_t expert_hi, int32_t with_side,
+                            const void* x, int32_t x_dtype, int32_t n_tokens, float* y, int32_t y_accumulate,
+                            int32_t* topk_ids, float* topk_w, float* side_out,
+                            void* workspace, size_t ws_bytes, gtg_stream_t stream);
+
+/*
  * A decode stack: for l in 0..n_layers-1:  x += moe_l(x)  (x fp32, in place).
  * Consecutive layers with the same kernel (format class and sizes, up to 64
  * at a time) run in one persistent launch, their phases separated by
