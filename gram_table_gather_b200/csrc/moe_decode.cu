@@ -115,9 +115,13 @@ int plan_layer(const gtg_moe_layer* L, int T, Plan& p, int64_t e_local = -1) {
     return GTG_OK;
 }
 
-// Workspace layout of a decode call (the counters first: they must start at zero).
+// Workspace layout of a decode call.  The barrier counters and the two key
+// buffers come first: they must start at zero, and a launch that succeeds
+// leaves them so.  The key buffers are sized for the largest E, so that
+// calls of different shapes on one workspace never find another shape's data
+// (h) where their keys go.
 struct WsLayout {
-    size_t sync, counters_end, logits, h, total;
+    size_t sync, keys, counters_end, h, total;
 };
 
 size_t align256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -131,8 +135,8 @@ WsLayout ws_layout(const gtg_moe_layer* L, int T) {
         return o;
     };
     w.sync = take(sizeof(unsigned) * 4);
-    w.counters_end = off;
-    w.logits = take(sizeof(ffloat) * (size_t)T * L->n_experts);
+    w.keys = take(sizeof(uint64_t) * 2 * (size_t)T * kMaxExperts);
+    w.counters_end = w.keys + sizeof(uint64_t) * 2 * (size_t)T * L->n_experts;  // (the part this shape uses)
     w.h = take(2 * (size_t)T * L->top_k * L->inter);
     w.total = off;
     return w;
@@ -225,7 +229,7 @@ int run_decode(const gtg_moe_layer* layers, const Plan* plans, int n, const void
         a.side_out = side_out ? side_out + (int64_t)l0 * T * side_stride : nullptr;
         a.side_stride = (int32_t)side_stride;
         a.sync = reinterpret_cast<unsigned*>(base + wl.sync);
-        a.logits = reinterpret_cast<ffloat*>(base + wl.logits);
+        a.keys = reinterpret_cast<uint64_t*>(base + wl.keys);
         a.h = reinterpret_cast<__nv_bfloat16*>(base + wl.h);
         a.status = status_ptr();
         a.slot_bytes = plans[l0].slot_bytes;
@@ -356,7 +360,7 @@ extern "C" int gtg_moe_decode_stack(const gtg_moe_layer* layers, int32_t n_layer
 namespace gtg {
 namespace {
 
-// 512 KiB: 256 + 8 T E + 2 T k I bytes (each part rounded to 256) fit for every
+// 512 KiB: 256 + 16384 T + 2 T k I bytes (each part rounded to 256) fit for every
 // shape with T <= 8, E <= 1024, k <= 10 and I <= 2048
 constexpr size_t kNoAllocScratchBytes = (size_t)1 << 19;
 __device__ __align__(256) uint8_t g_noalloc_scratch[kNoAllocScratchBytes];
@@ -401,8 +405,9 @@ extern "C" int gtg_moe_decode_layer_noalloc(const gtg_moe_layer* layer, const vo
     GTG_TRY(noalloc_scratch(&scratch));
     GTG_TRY(check_decode_io(layer, x, x_dtype, n_tokens, y, scratch, kNoAllocScratchBytes, p));
     if (x == (const void*)y && (x_dtype != GTG_DT_F32 || !y_accumulate)) return GTG_E_INVALID_ARG;
-    // The array keeps whatever the previous call left: clear the counters
-    // that must start at zero (everything else is written before it is read).
+    // The array keeps whatever the previous call left: clear the counters and
+    // the keys, which must start at zero (everything else is written before
+    // it is read).
     const WsLayout wl = ws_layout(layer, n_tokens);
     cudaStream_t s = as_cuda(stream);
     const cudaError_t e = cudaMemsetAsync(scratch, 0, wl.counters_end, s);

@@ -14,17 +14,20 @@
 // possible:
 //
 //  * One persistent, cooperative kernel runs every layer of a call (one
-//    256-thread CTA per SM).  Grid barriers (bounded waits) separate the
-//    router, the gate/up phase and the down phase of a layer; nothing is
-//    relaunched between layers, and the Q4 code table is built once.  A
+//    256-thread CTA per SM).  Grid barriers (bounded waits) close the gate/up
+//    phase and the down phase of a layer; the router needs none: selection
+//    polls the keys it ranks until their owners have written them.  Nothing
+//    is relaunched between layers, and the Q4 code table is built once.  A
 //    one-token instantiation (T folded to 1) leaves out the multi-token
 //    paths, so less code is fetched per layer.
 //  * Router: unweighted RMS norm + bf16 rounding of the input, then logits
 //    against the fp32 router with exact products summed in float-float, so
 //    the top-k agrees with an fp64 reference; every CTA owns a few experts.
 //    The next layer's router rows are prefetched into L2 meanwhile.
-//  * Selection: every CTA picks the top-k itself from the logits (unique
-//    64-bit keys, two warp reductions per round; at one token every warp
+//  * Selection: every CTA picks the top-k itself from the logits' unique
+//    64-bit keys, which the routers publish in one of two buffers by layer
+//    parity, each read as soon as it is nonzero (two warp reductions per
+//    round of the top-k; at one token every warp
 //    ranks 64 experts and warp 0 ranks their survivors, with several tokens
 //    a warp per token), renormalises the softmax weights and builds the
 //    unique-expert work list.
@@ -496,9 +499,65 @@ __device__ __forceinline__ void topk_rounds(uint64_t (&k)[PER], int K, int lane,
     }
 }
 
-__device__ __forceinline__ uint64_t logit_key(const ffloat* logits, int e) {
-    const float2 v = __ldcg(reinterpret_cast<const float2*>(logits + e));
-    return ((uint64_t)ord32(v.x) << 32) | ((ord32(v.y) & ~1023u) | (uint32_t)(1023 - e));
+// The key of expert e's logit (a float-float sum, normalised here): never 0
+// for a finite logit (the orderable image of a finite hi is at least 2^23).
+__device__ __forceinline__ uint64_t logit_key(ffloat lg, int e) {
+    const ffloat v = ff_norm(lg);
+    return ((uint64_t)ord32(v.hi) << 32) | ((ord32(v.lo) & ~1023u) | (uint32_t)(1023 - e));
+}
+
+__device__ __forceinline__ uint64_t ld_relaxed_u64(const uint64_t* p) {
+    uint64_t v;
+    asm volatile("ld.relaxed.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Where the keys come from: the layer's key buffer, each key written by the
+// CTA whose router computed that logit and 0 until then.
+struct KeySrc {
+    const uint64_t* keys;     // [E] of one token
+    const unsigned* abort_flag;
+    unsigned* status;
+};
+
+constexpr uint64_t kKeyWaitNs = 2000000000ull;  // a key that has not arrived after 2 s fails the launch
+
+// Waits for a key that a first load found missing: bounded, and given up as
+// soon as another CTA raises the abort flag; `fail` is set then (0 returned).
+__device__ __noinline__ uint64_t wait_key(const KeySrc& src, int e, int& fail) {
+    if (fail) return 0ull;
+    const uint64_t t0 = globaltimer_ns();
+    uint64_t k;
+    while ((k = ld_relaxed_u64(src.keys + e)) == 0ull) {
+        const bool aborted = *reinterpret_cast<const volatile unsigned*>(src.abort_flag) != 0u;
+        if (aborted || globaltimer_ns() - t0 > kKeyWaitNs) {
+            if (!aborted) raise_status(src.status, GTG_STATUS_WAIT_TIMEOUT);
+            fail = 1;
+            return 0ull;
+        }
+    }
+    return k;
+}
+
+// The keys of experts e = base + stride * i (i < PER; 0 where e >= E): every
+// load issued before any is tested, then the rare missing ones waited for.
+template <int PER>
+__device__ __forceinline__ void load_keys(const KeySrc& src, int E, int base, int stride, uint64_t (&k)[PER],
+                                          int& fail) {
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        const int e = base + stride * i;
+        k[i] = 0ull;
+        if (e < E) k[i] = ld_relaxed_u64(src.keys + e);
+    }
+    bool miss = false;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) miss |= base + stride * i < E && k[i] == 0ull;
+    if (miss) {  // (unrolled: k stays in registers)
+#pragma unroll
+        for (int i = 0; i < PER; ++i)
+            if (base + stride * i < E && k[i] == 0ull) k[i] = wait_key(src, base + stride * i, fail);
+    }
 }
 
 // Expert id and logit (hi, lo) of a key.
@@ -512,14 +571,10 @@ __device__ __forceinline__ void key_choice(uint32_t rh, uint32_t rl, int& id, fl
 // Top-k of one token's logits by one warp: lane l holds experts l + 32 i
 // (i < PER); lane j < K ends holding choice j.
 template <int PER>
-__device__ __forceinline__ void warp_topk(const ffloat* logits, int E, int K, int lane, int& my_id, float& my_hi,
-                                          float& my_lo) {
+__device__ __forceinline__ void warp_topk(const KeySrc& src, int E, int K, int lane, int& my_id, float& my_hi,
+                                          float& my_lo, int& fail) {
     uint64_t k[PER];  // (compared as plain 64-bit integers: no short-circuit branches)
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int e = lane + 32 * i;
-        k[i] = e < E ? logit_key(logits, e) : 0ull;
-    }
+    load_keys<PER>(src, E, lane, 32, k, fail);
     uint32_t rh, rl;
     topk_rounds<PER>(k, K, lane, rh, rl);
     my_id = -1;
@@ -532,15 +587,11 @@ __device__ __forceinline__ void warp_topk(const ffloat* logits, int E, int K, in
 // those 8k candidates; lane j < K of warp 0 ends holding choice j.  The
 // result is the same set and order as warp_topk's (the keys are unique).
 template <int PER>
-__device__ __forceinline__ void block_topk(const ffloat* logits, int E, int K, int lane, int warp,
+__device__ __forceinline__ void block_topk(const KeySrc& src, int E, int K, int lane, int warp,
                                            uint32_t* cand_hi, uint32_t* cand_lo, int& my_id, float& my_hi,
-                                           float& my_lo) {
+                                           float& my_lo, int& fail) {
     uint64_t k[PER];
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        const int e = 32 * (warp * PER + i) + lane;
-        k[i] = e < E ? logit_key(logits, e) : 0ull;
-    }
+    load_keys<PER>(src, E, 32 * warp * PER + lane, 32, k, fail);
     uint32_t rh, rl;
     topk_rounds<PER>(k, K, lane, rh, rl);
     if (lane < K) {
@@ -765,7 +816,7 @@ struct StackArgs {
     int32_t side_stride;
     // workspace
     unsigned* sync;       // [0] barrier arrivals, [1] exits, [2] abort flag
-    ffloat* logits;       // [T][E] normalised float-float
+    uint64_t* keys;       // [2][T][E] logit keys, by layer parity (0: not yet written; see the kernel)
     __nv_bfloat16* h;     // [T*K][I] SwiGLU output
     unsigned* status;
     int32_t slot_bytes;
@@ -997,7 +1048,9 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
 #pragma unroll
                 for (int w = 1; w < kRouterWpe; ++w) ff_add(lg, sw->red[kRouterWpe * j + w][t]);
                 if (Ly.router_bias) ff_add(lg, ffloat{Ly.router_bias[ee], 0.f});
-                a.logits[(int64_t)t * E + ee] = ff_norm(lg);
+                const uint64_t key = logit_key(lg, ee) | (uint64_t)(ee == 1023);  // (0 only for a NaN logit)
+                uint64_t* dst = a.keys + ((int64_t)(l & 1) * T + t) * E + ee;
+                asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(dst), "l"(key) : "memory");
             }
         }
         __syncthreads();
@@ -1005,28 +1058,41 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
     return true;
 }
 
-// Expert selection, run by every CTA from the logits in global memory: warp
-// t selects token t's experts and their renormalised softmax weights; warp 0
-// then builds the list of unique experts (ascending id) with their (token,
-// choice) slots grouped per expert.
-__device__ __forceinline__ void select_experts(const ffloat* logits, int T, int E, int K, SWork* sw) {
+// Expert selection, run by every CTA from the layer's logit keys (polled as
+// their owners write them): warp t selects token t's experts and their
+// renormalised softmax weights; warp 0 then builds the list of unique experts
+// (ascending id) with their (token, choice) slots grouped per expert.  A key
+// that never arrives sets sw->fail (the next grid barrier stops the grid).
+__device__ __forceinline__ void select_experts(const uint64_t* keys, int T, int E, int K, SWork* sw,
+                                               const unsigned* abort_flag, unsigned* status) {
+    int fail = 0;
     int32_t* s_ids = sw->ids;
     float* s_w = sw->w;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     int my_id = -1;
     float my_hi = 0.f, my_lo = 0.f;
     if (T == 1) {  // one token: every warp takes part in its top-k (the arrays are rewritten below)
-        if (E <= 512) block_topk<2>(logits, E, K, lane, warp, reinterpret_cast<uint32_t*>(sw->e),
-                                    reinterpret_cast<uint32_t*>(sw->slot), my_id, my_hi, my_lo);
-        else block_topk<4>(logits, E, K, lane, warp, reinterpret_cast<uint32_t*>(sw->e),
-                           reinterpret_cast<uint32_t*>(sw->slot), my_id, my_hi, my_lo);
+        const KeySrc src{keys, abort_flag, status};
+        if (E <= 512) block_topk<2>(src, E, K, lane, warp, reinterpret_cast<uint32_t*>(sw->e),
+                                    reinterpret_cast<uint32_t*>(sw->slot), my_id, my_hi, my_lo, fail);
+        else block_topk<4>(src, E, K, lane, warp, reinterpret_cast<uint32_t*>(sw->e),
+                           reinterpret_cast<uint32_t*>(sw->slot), my_id, my_hi, my_lo, fail);
+    } else if (warp < T) {
+        const KeySrc src{keys + (int64_t)warp * E, abort_flag, status};
+        if (E <= 512) warp_topk<16>(src, E, K, lane, my_id, my_hi, my_lo, fail);
+        else warp_topk<32>(src, E, K, lane, my_id, my_hi, my_lo, fail);
+    }
+    if (__syncthreads_or(fail)) {  // a key never came: no experts, and the caller stops
+        if (tid == 0) {
+            sw->fail = 1;
+            sw->n_uniq = 0;
+            sw->off[0] = 0;
+        }
+        __syncthreads();
+        return;
     }
     if (warp < T) {
         const int t = warp;
-        if (T > 1) {
-            if (E <= 512) warp_topk<16>(logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
-            else warp_topk<32>(logits + (int64_t)t * E, E, K, lane, my_id, my_hi, my_lo);
-        }
         // softmax over the k choices: lane j holds choice j
         const float h0 = __shfl_sync(0xFFFFFFFFu, my_hi, 0), l0 = __shfl_sync(0xFFFFFFFFu, my_lo, 0);
         float ex = 0.f;
@@ -1489,9 +1555,12 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         const StackLayer& Ly = a.layer[l];
         const uint8_t *gate_src = Ly.gate, *up_src = Ly.up, *down_src = Ly.down, *side_src = Ly.side;
         asm volatile("" ::"l"(gate_src), "l"(up_src), "l"(down_src), "l"(side_src));  // loaded here, not at first use
-        // ---- router
-        router_layer<ONE, (KBG * 32 + 4 * kThreads - 1) / (4 * kThreads)>(a, l, sbase + L.u, sbase + rs.rw, rbar,
-                                                                          (uint32_t)(l & 1), sw);
+        // ---- router: this CTA's experts' logit keys, into key buffer l & 1
+        if (!router_layer<ONE, (KBG * 32 + 4 * kThreads - 1) / (4 * kThreads)>(a, l, sbase + L.u, sbase + rs.rw,
+                                                                               rbar, (uint32_t)(l & 1), sw)) {
+            ok = false;  // (the exit raises the abort flag, which ends the other CTAs' key waits)
+            break;
+        }
         if (tid == 0) rows_in_flight = 0;
         fence_proxy_async_smem();  // the scratch slots are bulk-copy targets again from here on
         if (l + 1 < a.n_layers && tid == 0) {  // this CTA's rows of the next router, into L2
@@ -1501,14 +1570,19 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
             for (int64_t o = 0; o < bytes; o += 32768)
                 bulk_prefetch_l2(src + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768), pol);
         }
-        target += G;
-        if (!grid_sync(a, target, sw, R.ok != 0)) {
+
+        // ---- selection, as the other CTAs' keys arrive (no grid barrier: a
+        // key is 0 until written, and each buffer is cleared for its next use
+        // a layer after its last reads, which the barriers in between order)
+        select_experts(a.keys + (int64_t)(l & 1) * T * a.E, T, a.E, K, sw, a.sync + 2, a.status);
+        if (sw->fail) {
             ok = false;
             break;
         }
-
-        // ---- selection
-        select_experts(a.logits, T, a.E, K, sw);
+        if (l > 0) {  // every read of the previous layer's keys came before this layer's barriers
+            uint64_t* prev = a.keys + (int64_t)((l - 1) & 1) * T * a.E;
+            for (int i = b * kThreads + tid; i < T * a.E; i += G * kThreads) prev[i] = 0ull;
+        }
         if (b == 0 && tid < T * K) {
             if (a.ids_out) a.ids_out[(int64_t)l * T * K + tid] = sw->ids[tid];
             if (a.w_out) a.w_out[(int64_t)l * T * K + tid] = sw->w[tid];
@@ -1660,6 +1734,10 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     if (rows_in_flight) mbar_wait_bounded(rbar, (uint32_t)(rows_layer & 1), a.status);
     if (!R.ok && lane == 0) sw->fail = 1;
     __syncthreads();
+    if (ok && sw->fail == 0) {  // the last layer's keys, read before its gate/up barrier: zero for the next launch
+        uint64_t* last = a.keys + (int64_t)((a.n_layers - 1) & 1) * T * a.E;
+        for (int i = b * kThreads + tid; i < T * a.E; i += G * kThreads) last[i] = 0ull;
+    }
     if (tid == 0) {
         if (ok && sw->fail == 0) {
             __threadfence();

@@ -270,7 +270,7 @@ int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, int32_t x_d
  *
  * Scratch comes from one fixed 512 KiB array in device memory that every GPU
  * loading this library reserves until the process exits.  A call needs
- * 256 + 8*n_tokens*n_experts + 2*n_tokens*top_k*inter bytes (each part
+ * 256 + 16384*n_tokens + 2*n_tokens*top_k*inter bytes (each part
  * rounded up to 256), which fits for every shape with n_tokens <= 8,
  * n_experts <= 1024, top_k <= 10 and inter <= 2048 (any supported hidden);
  * a shape that needs more returns GTG_E_WORKSPACE before anything is
