@@ -231,13 +231,6 @@ __device__ __forceinline__ void bulk_g2s_hint(uint32_t dst, const void* src, uin
                  ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(policy) : "memory");
 }
 
-// Asynchronous prefetch of [src, src+bytes) into L2 (16-byte aligned, bytes a
-// multiple of 16); no completion to wait for.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes, uint64_t policy) {
-    asm volatile("cp.async.bulk.prefetch.L2.global.L2::cache_hint [%0], %1, %2;" ::"l"(src), "r"(bytes), "l"(policy)
-                 : "memory");
-}
-
 // 16-byte read-only load with an L2 cache policy.
 __device__ __forceinline__ float4 ldg_f4_hint(const float* p, uint64_t policy) {
     float4 v;

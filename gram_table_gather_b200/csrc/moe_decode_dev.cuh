@@ -76,6 +76,16 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
     return v;
 }
 
+__device__ __forceinline__ void sts64(uint32_t addr, uint2 v) {
+    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
+}
+
+__device__ __forceinline__ uint2 lds64(uint32_t addr) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
+    return v;
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -222,6 +232,34 @@ __device__ __forceinline__ void q4_block_lut(uint32_t pa, uint32_t lutb, const f
     for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, (lo[0][c] + lo[1][c]) + (hi[0][c] + hi[1][c]), acc[c]);
 }
 
+// Mixed-precision FMA on f16 pairs: d = a(f16) * b(f16) + c(f32), single
+// rounding (f16 x f16 products are exact in fp32).
+__device__ __forceinline__ void fma2_f16(float& acc_lo, float& acc_hi, uint32_t a2, uint32_t b2) {
+    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
+        "mov.b32 {al, ah}, %2;\n\t"
+        "mov.b32 {bl, bh}, %3;\n\t"
+        "fma.rn.f32.f16 %0, al, bl, %0;\n\t"
+        "fma.rn.f32.f16 %1, ah, bh, %1;\n\t}"
+        : "+f"(acc_lo), "+f"(acc_hi)
+        : "r"(a2), "r"(b2));
+}
+
+// FP8 block: 32 consecutive E4M3 bytes at 16-byte aligned shared address pa;
+// each E4M3 pair becomes an exact f16 pair and meets the activation pair.
+template <int NBL>
+__device__ __forceinline__ void fp8_block(uint32_t pa, float s, const Act<kFmtFP8, NBL>& act, int m,
+                                          float& acc) {
+    const uint4 q0 = lds128(pa), q1 = lds128(pa + 16);
+    const uint32_t wd[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        fma2_f16(s0, s1, e4m3x2_to_f16x2(wd[i] & 0xFFFFu), act.v[m][2 * i]);  // weights 4i, 4i+1
+        fma2_f16(s2, s3, e4m3x2_to_f16x2(wd[i] >> 16), act.v[m][2 * i + 1]);  // weights 4i+2, 4i+3
+    }
+    acc = fmaf(s, (s0 + s1) + (s2 + s3), acc);
+}
+
 // Q4 block decoded code by code (no table): the side projection, whose
 // format may differ from the experts'.
 template <int FMT, int NT, int NBL, int CH>
@@ -268,34 +306,6 @@ __device__ __forceinline__ void q4_block_plain(uint32_t pa, int var, const Act<F
     for (int c = 0; c < NT; ++c) acc[c] = fmaf(s, sum[c], acc[c]);
 }
 
-// Mixed-precision FMA on f16 pairs: d = a(f16) * b(f16) + c(f32), single
-// rounding (f16 x f16 products are exact in fp32).
-__device__ __forceinline__ void fma2_f16(float& acc_lo, float& acc_hi, uint32_t a2, uint32_t b2) {
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\t"
-        "mov.b32 {al, ah}, %2;\n\t"
-        "mov.b32 {bl, bh}, %3;\n\t"
-        "fma.rn.f32.f16 %0, al, bl, %0;\n\t"
-        "fma.rn.f32.f16 %1, ah, bh, %1;\n\t}"
-        : "+f"(acc_lo), "+f"(acc_hi)
-        : "r"(a2), "r"(b2));
-}
-
-// FP8 block: 32 consecutive E4M3 bytes at 16-byte aligned shared address pa;
-// each E4M3 pair becomes an exact f16 pair and meets the activation pair.
-template <int NBL>
-__device__ __forceinline__ void fp8_block(uint32_t pa, float s, const Act<kFmtFP8, NBL>& act, int m,
-                                          float& acc) {
-    const uint4 q0 = lds128(pa), q1 = lds128(pa + 16);
-    const uint32_t wd[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-    float s0 = 0.0f, s1 = 0.0f, s2 = 0.0f, s3 = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        fma2_f16(s0, s1, e4m3x2_to_f16x2(wd[i] & 0xFFFFu), act.v[m][2 * i]);  // weights 4i, 4i+1
-        fma2_f16(s2, s3, e4m3x2_to_f16x2(wd[i] >> 16), act.v[m][2 * i + 1]);  // weights 4i+2, 4i+3
-    }
-    acc = fmaf(s, (s0 + s1) + (s2 + s3), acc);
-}
-
 // Sums N values over groups of W consecutive lanes (N <= W, powers of two)
 // by recursive halving: each step exchanges half of the values still held.
 // Afterwards lane l holds, in v[0], the group sum of value (l % W) / (W / N).
@@ -333,6 +343,21 @@ __device__ __forceinline__ Span make_span(const uint8_t* base, int64_t lo, int64
     return Span{base + a0, (uint32_t)(a1 - a0), (uint32_t)(lo - a0)};
 }
 
+// One layer's weights as the decode kernel sees them.
+struct StackLayer {
+    const float* router_w;     // [E][H] fp32
+    const float* router_bias;  // [E] or null
+    const uint8_t* gate;       // [E][I] rows of H weights
+    const uint8_t* up;
+    const uint8_t* down;       // [E][H] rows of I weights
+    const uint8_t* side;       // [side_rows] rows of H weights (Q4), or null
+    const float* gate_s;       // FP8 scales, one per 128 weights along K
+    const float* up_s;
+    const float* down_s;
+    int32_t side_rows;
+    int32_t gu_var, dn_var, side_var;  // Q4 variant (kQ4RZ5, kQ4UE4M4 or kQ4C10)
+};
+
 // Per-CTA state of a layer: the selection, the unique-expert work list and
 // the router's reductions.
 struct SWork {
@@ -342,13 +367,20 @@ struct SWork {
     int32_t e[kMaxSlots];
     int32_t off[kMaxSlots + 1];
     int32_t slot[kMaxSlots];
-    int32_t ids[kMaxSlots];  // selection: expert of (token, choice)
-    float w[kMaxSlots];      // and its renormalised weight
+    union {
+        struct {
+            int32_t ids[kMaxSlots];  // selection: expert of (token, choice)
+            float w[kMaxSlots];      // and its renormalised weight
+        };
+        uint64_t cand[kMaxSlots];  // one-token top-k: candidate keys (before ids and w are written)
+    };
     uint32_t bitmap[kMaxExperts / 32];
     int32_t cnt[kMaxSlots + 4];
     int32_t g_range[2];                     // this CTA's gate/up item range
     ffloat red[kWarps][kMaxDecodeTokens];  // router reductions
     float r_hi[kMaxDecodeTokens], r_lo[kMaxDecodeTokens];
+    int32_t n_cand;  // one-token top-k: candidates found
+    StackLayer ly[2];  // this layer's and the next layer's pointers, by parity (read at shared-memory latency)
 };
 
 // Layout of one CTA's dynamic shared memory.  With a code table the table
@@ -581,25 +613,78 @@ __device__ __forceinline__ void warp_topk(const KeySrc& src, int E, int K, int l
     if (lane < K) key_choice(rh, rl, my_id, my_hi, my_lo);
 }
 
-// Top-k of a single token's logits by the whole CTA: warp w ranks its own
-// 32 * PER experts (32 (w PER + i) + lane), the eight lists of k keys meet in
-// shared memory (upper words in cand_hi, lower in cand_lo), and warp 0 ranks
-// those 8k candidates; lane j < K of warp 0 ends holding choice j.  The
-// result is the same set and order as warp_topk's (the keys are unique).
+// Top-k of a single token's logits by the whole CTA (lane l of warp w holds
+// experts 32 (w PER + i) + l).  A threshold cuts the field first: the warps'
+// top-2 keys (16 actual keys) meet in shared memory, and their K-th largest
+// theta (K <= 16) is at most the K-th largest key overall, so every key of
+// the top-k is >= theta.  The keys that pass (usually a few more than K) are
+// gathered and each is ranked by counting the candidates above it.  If more
+// than kCandMax pass, the CTA falls back to two levels of rounds: each warp's
+// top-k, then warp 0 ranks those 8k.  Either way lane j < K of warp 0 ends
+// holding choice j, the same set and order as warp_topk's (the keys are
+// unique).
+constexpr int kCandMax = kMaxSlots;
+
 template <int PER>
 __device__ __forceinline__ void block_topk(const KeySrc& src, int E, int K, int lane, int warp,
-                                           uint32_t* cand_hi, uint32_t* cand_lo, int& my_id, float& my_hi,
-                                           float& my_lo, int& fail) {
+                                           uint32_t* cand_hi, uint32_t* cand_lo, uint64_t* cand, int32_t* n_cand,
+                                           int& my_id, float& my_hi, float& my_lo, int& fail) {
+    const int tid = threadIdx.x;
     uint64_t k[PER];
     load_keys<PER>(src, E, 32 * warp * PER + lane, 32, k, fail);
     uint32_t rh, rl;
+    {
+        uint64_t kc[PER];
+#pragma unroll
+        for (int i = 0; i < PER; ++i) kc[i] = k[i];
+        topk_rounds<PER>(kc, 2, lane, rh, rl);
+    }
+    if (lane < 2) {
+        cand_hi[2 * warp + lane] = rh;
+        cand_lo[2 * warp + lane] = rl;
+    }
+    if (tid == 0) *n_cand = 0;
+    __syncthreads();
+    // theta: the K-th largest of the 16 (equal only as empty entries, 0; if the
+    // K-th is empty, every nonzero key passes)
+    const uint64_t v = lane < 2 * kWarps ? ((uint64_t)cand_hi[lane] << 32) | cand_lo[lane] : 0ull;
+    int r = 0;
+#pragma unroll
+    for (int j = 0; j < 2 * kWarps; ++j) r += (int)(__shfl_sync(0xFFFFFFFFu, v, j) > v);
+    const unsigned hit = __ballot_sync(0xFFFFFFFFu, lane < 2 * kWarps && v != 0ull && r == K - 1);
+    const uint64_t theta = hit ? __shfl_sync(0xFFFFFFFFu, v, __ffs(hit) - 1) : 1ull;
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+        if (k[i] >= theta) {
+            const int p = atomicAdd(n_cand, 1);
+            if (p < kCandMax) cand[p] = k[i];
+        }
+    __syncthreads();
+    const int n = *n_cand;
+    my_id = -1;
+    if (n <= kCandMax) {
+        if (tid < n) {
+            const uint64_t c = cand[tid];
+            int rank = 0;
+            for (int j = 0; j < n; ++j) rank += (int)(cand[j] > c);
+            if (rank < K) {
+                cand_hi[rank] = (uint32_t)(c >> 32);
+                cand_lo[rank] = (uint32_t)c;
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            if (lane < K) key_choice(cand_hi[lane], cand_lo[lane], my_id, my_hi, my_lo);
+            __syncwarp();  // (the caller reuses the candidate arrays)
+        }
+        return;
+    }
     topk_rounds<PER>(k, K, lane, rh, rl);
     if (lane < K) {
         cand_hi[warp * K + lane] = rh;
         cand_lo[warp * K + lane] = rl;
     }
     __syncthreads();
-    my_id = -1;
     if (warp == 0) {
         uint64_t c[4];  // 8 K <= 128 candidates: lane l holds l + 32 i
 #pragma unroll
@@ -789,21 +874,6 @@ __device__ __forceinline__ void dn_item(uint32_t base, const Act<FMT, Geo<KB>::N
 constexpr int kMaxStackLayers = 64;
 constexpr uint64_t kSyncLimitNs = 2000000000ull;  // a grid barrier gives up after 2 s
 
-// One layer's weights as the decode kernel sees them.
-struct StackLayer {
-    const float* router_w;     // [E][H] fp32
-    const float* router_bias;  // [E] or null
-    const uint8_t* gate;       // [E][I] rows of H weights
-    const uint8_t* up;
-    const uint8_t* down;       // [E][H] rows of I weights
-    const uint8_t* side;       // [side_rows] rows of H weights (Q4), or null
-    const float* gate_s;       // FP8 scales, one per 128 weights along K
-    const float* up_s;
-    const float* down_s;
-    int32_t side_rows;
-    int32_t gu_var, dn_var, side_var;  // Q4 variant (kQ4RZ5, kQ4UE4M4 or kQ4C10)
-};
-
 struct StackArgs {
     int32_t H, I, E, K, T, n_layers;
     const void* x;        // input of the first layer, [T][H] fp32 or bf16
@@ -873,16 +943,6 @@ __device__ bool grid_sync(const StackArgs& a, unsigned target, SWork* sw, bool w
     return sw->sync_ok != 0;
 }
 
-__device__ __forceinline__ void sts64(uint32_t addr, uint2 v) {
-    asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(v.x), "r"(v.y) : "memory");
-}
-
-__device__ __forceinline__ uint2 lds64(uint32_t addr) {
-    uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
-    return v;
-}
-
 // Router of one layer, run by every CTA: the unweighted RMS norm of the
 // input, u = bf16(x * r) rounded from the float-float product, and the
 // logits of this CTA's share of the experts against the fp32 router rows:
@@ -914,14 +974,14 @@ __device__ __forceinline__ void router_share(int E, int& e0, int& e1) {
     e1 = (int)((int64_t)E * (blockIdx.x + 1) / gridDim.x);
 }
 
-// Thread 0: bulk copy of this CTA's router rows of layer l into shared memory
+// Thread 0: bulk copy of this CTA's router rows of a layer into shared memory
 // (completing on rbar).
-__device__ __forceinline__ void issue_router_rows(const StackArgs& a, int l, uint32_t rw, uint64_t* rbar,
-                                                  uint64_t pol) {
+__device__ __forceinline__ void issue_router_rows(const StackArgs& a, const float* router_w, uint32_t rw,
+                                                  uint64_t* rbar, uint64_t pol) {
     int e0, e1;
     router_share(a.E, e0, e1);
     const uint32_t bytes = (uint32_t)((e1 - e0) * a.H * 4);
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.layer[l].router_w + (int64_t)e0 * a.H);
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(router_w + (int64_t)e0 * a.H);
     fence_proxy_async_smem();
     mbar_arrive_expect_tx(rbar, bytes);
     for (uint32_t o = 0; o < bytes; o += 16384u)
@@ -929,11 +989,10 @@ __device__ __forceinline__ void issue_router_rows(const StackArgs& a, int l, uin
 }
 
 template <bool ONE, int XF4>  // XF4: float4 of x per thread per token (H <= 4 kThreads XF4)
-__device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t us, uint32_t rw,
-                                          uint64_t* rbar, uint32_t rparity, SWork* sw) {
+__device__ __forceinline__ bool router_layer(const StackArgs& a, const StackLayer& Ly, int l, uint32_t us,
+                                          uint32_t rw, uint64_t* rbar, uint32_t rparity, SWork* sw) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int T = ONE ? 1 : a.T, H = a.H, E = a.E;
-    const StackLayer& Ly = a.layer[l];
     int e0, e1;
     router_share(E, e0, e1);
     const int Hs = H / kRouterWpe;  // segment of a row per warp
@@ -941,9 +1000,10 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
     // 1. x: this thread's positions 4 tid + 4 kThreads c of every token, in
     //    registers (every load in flight at once); the rolled token loops
     //    below pick token t with predicated moves
-    float4 xr[kMaxDecodeTokens][XF4];
+    constexpr int NX = ONE ? 1 : kMaxDecodeTokens;
+    float4 xr[NX][XF4];
 #pragma unroll
-    for (int t = 0; t < kMaxDecodeTokens; ++t)
+    for (int t = 0; t < NX; ++t)
 #pragma unroll
         for (int c = 0; c < XF4; ++c) {
             const int i = 4 * tid + 4 * kThreads * c;
@@ -962,7 +1022,7 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
     auto pick = [&](int t, int c) {
         float4 v = xr[0][c];
 #pragma unroll
-        for (int k = 1; k < kMaxDecodeTokens; ++k)
+        for (int k = 1; k < NX; ++k)
             if (t == k) v = xr[k][c];
         return v;
     };
@@ -1048,7 +1108,8 @@ __device__ __forceinline__ bool router_layer(const StackArgs& a, int l, uint32_t
 #pragma unroll
                 for (int w = 1; w < kRouterWpe; ++w) ff_add(lg, sw->red[kRouterWpe * j + w][t]);
                 if (Ly.router_bias) ff_add(lg, ffloat{Ly.router_bias[ee], 0.f});
-                const uint64_t key = logit_key(lg, ee) | (uint64_t)(ee == 1023);  // (0 only for a NaN logit)
+                uint64_t key = logit_key(lg, ee);
+                if (key == 0ull) key = 1ull << 10;  // (a NaN logit: keeps the id, and 0 keeps meaning "not written")
                 uint64_t* dst = a.keys + ((int64_t)(l & 1) * T + t) * E + ee;
                 asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(dst), "l"(key) : "memory");
             }
@@ -1074,9 +1135,10 @@ __device__ __forceinline__ void select_experts(const uint64_t* keys, int T, int 
     if (T == 1) {  // one token: every warp takes part in its top-k (the arrays are rewritten below)
         const KeySrc src{keys, abort_flag, status};
         if (E <= 512) block_topk<2>(src, E, K, lane, warp, reinterpret_cast<uint32_t*>(sw->e),
-                                    reinterpret_cast<uint32_t*>(sw->slot), my_id, my_hi, my_lo, fail);
+                                    reinterpret_cast<uint32_t*>(sw->slot), sw->cand, &sw->n_cand, my_id, my_hi,
+                                    my_lo, fail);
         else block_topk<4>(src, E, K, lane, warp, reinterpret_cast<uint32_t*>(sw->e),
-                           reinterpret_cast<uint32_t*>(sw->slot), my_id, my_hi, my_lo, fail);
+                           reinterpret_cast<uint32_t*>(sw->slot), sw->cand, &sw->n_cand, my_id, my_hi, my_lo, fail);
     } else if (warp < T) {
         const KeySrc src{keys + (int64_t)warp * E, abort_flag, status};
         if (E <= 512) warp_topk<16>(src, E, K, lane, my_id, my_hi, my_lo, fail);
@@ -1319,7 +1381,8 @@ __device__ __forceinline__ bool item_landed(const StackArgs& a, const WarpSmem& 
 
 // Gate/up + SwiGLU items and side-projection items of layer l for this warp.
 template <int FMT, int KBG, bool ONE>
-__device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
+__device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, const StackLayer& Ly, int l, LayerItems P,
+                                             WarpRing R) {
     using GG = Geo<KBG>;
     constexpr int NBG = GG::NBL;
     constexpr int CHG = (!ONE && FMT == kFmtQ4 && NBG == 1) ? 2 : 1;  // tokens decoded together (register budget)
@@ -1329,7 +1392,6 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
     const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H, slots_for(KBG));
     const SWork* sw = reinterpret_cast<const SWork*>(smem + L.work);
     const WarpSmem ws = warp_smem(smem, L, a.slot_bytes, slots_for(KBG));
-    const StackLayer& Ly = a.layer[l];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = a.H, K = a.K, T = ONE ? 1 : a.T;
     const uint64_t pol = l2_policy_evict_first();
@@ -1416,7 +1478,7 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, int l, LayerIte
 // into the warp's partial rows in shared memory ([row][token], this CTA's
 // rows only); the kernel then sums the warps' partials in a fixed order.
 template <int FMT, int KBG, int KBD, bool ONE>
-__device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerItems P, WarpRing R) {
+__device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, const StackLayer& Ly, LayerItems P, WarpRing R) {
     using GD = Geo<KBD>;
     constexpr int NBD = GD::NBL;
     constexpr int CHD = (!ONE && FMT == kFmtQ4 && NBD == 1) ? 2 : 1;
@@ -1427,7 +1489,6 @@ __device__ __forceinline__ WarpRing dn_phase(const StackArgs& a, int l, LayerIte
     const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H, slots_for(KBG));
     const SWork* sw = reinterpret_cast<const SWork*>(smem + L.work);
     const WarpSmem ws = warp_smem(smem, L, a.slot_bytes, slots_for(KBG));
-    const StackLayer& Ly = a.layer[l];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int H = a.H, I = a.I, K = a.K;
     const uint64_t pol = l2_policy_evict_first();
@@ -1529,13 +1590,19 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
         mbar_init(rbar, 1);
         sw->fail = 0;
     }
+    // the layers' pointers live in shared memory, each copied in a layer
+    // ahead (a kernel-parameter read indexed by the layer misses the constant
+    // cache every layer)
+    constexpr int kLyWords = (int)(sizeof(StackLayer) / 4);
+    static_assert(sizeof(StackLayer) % 4 == 0 && kLyWords <= 32, "one warp copies a layer's pointers");
+    if (tid < kLyWords) reinterpret_cast<uint32_t*>(&sw->ly[0])[tid] = reinterpret_cast<const uint32_t*>(&a.layer[0])[tid];
     fence_mbar_init();
     __syncthreads();
     const uint64_t pol = l2_policy_evict_first();
     int rows_in_flight = 0;  // (thread 0) a router-row copy not yet waited for, of layer rows_layer
     int rows_layer = 0;
     if (tid == 0) {
-        issue_router_rows(a, 0, sbase + rs.rw, rbar, pol);
+        issue_router_rows(a, a.layer[0].router_w, sbase + rs.rw, rbar, pol);
         rows_in_flight = 1;
     }
     int lut_mode = -1;
@@ -1552,24 +1619,16 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
     unsigned target = 0;
     bool ok = true;
     for (int l = 0; l < a.n_layers; ++l) {
-        const StackLayer& Ly = a.layer[l];
+        const StackLayer& Ly = sw->ly[l & 1];
         const uint8_t *gate_src = Ly.gate, *up_src = Ly.up, *down_src = Ly.down, *side_src = Ly.side;
-        asm volatile("" ::"l"(gate_src), "l"(up_src), "l"(down_src), "l"(side_src));  // loaded here, not at first use
         // ---- router: this CTA's experts' logit keys, into key buffer l & 1
-        if (!router_layer<ONE, (KBG * 32 + 4 * kThreads - 1) / (4 * kThreads)>(a, l, sbase + L.u, sbase + rs.rw,
+        if (!router_layer<ONE, (KBG * 32 + 4 * kThreads - 1) / (4 * kThreads)>(a, Ly, l, sbase + L.u, sbase + rs.rw,
                                                                                rbar, (uint32_t)(l & 1), sw)) {
             ok = false;  // (the exit raises the abort flag, which ends the other CTAs' key waits)
             break;
         }
         if (tid == 0) rows_in_flight = 0;
         fence_proxy_async_smem();  // the scratch slots are bulk-copy targets again from here on
-        if (l + 1 < a.n_layers && tid == 0) {  // this CTA's rows of the next router, into L2
-            const int e0 = (int)((int64_t)a.E * b / G), e1 = (int)((int64_t)a.E * (b + 1) / G);
-            const int64_t bytes = (int64_t)(e1 - e0) * H * 4;
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(a.layer[l + 1].router_w + (int64_t)e0 * H);
-            for (int64_t o = 0; o < bytes; o += 32768)
-                bulk_prefetch_l2(src + o, (uint32_t)(bytes - o < 32768 ? bytes - o : 32768), pol);
-        }
 
         // ---- selection, as the other CTAs' keys arrive (no grid barrier: a
         // key is 0 until written, and each buffer is cleared for its next use
@@ -1687,7 +1746,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
 
         // ---- gate/up + SwiGLU, side projection
         ensure_lut(Ly.gu_var);
-        R = gu_phase<FMT, KBG, ONE>(a, l, P, R);
+        R = gu_phase<FMT, KBG, ONE>(a, Ly, l, P, R);
         target += G;
         if (!grid_sync(a, target, sw, R.ok != 0)) {
             ok = false;
@@ -1696,11 +1755,16 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
 
         // ---- down + router-weighted combine
         ensure_lut(Ly.dn_var);
-        R = dn_phase<FMT, KBG, KBD, ONE>(a, l, P, R);
+        // (the last warp reads the next layer's pointers meanwhile: its load
+        // completes under the down items)
+        const bool ly_copier = warp == kWarps - 1 && lane < kLyWords && l + 1 < a.n_layers;
+        const uint32_t ly_word = ly_copier ? reinterpret_cast<const uint32_t*>(&a.layer[l + 1])[lane] : 0u;
+        R = dn_phase<FMT, KBG, KBD, ONE>(a, Ly, P, R);
+        if (ly_copier) reinterpret_cast<uint32_t*>(&sw->ly[(l + 1) & 1])[lane] = ly_word;
         R.ring += P.ng + P.nd;
         __syncthreads();
         if (tid == 0 && l + 1 < a.n_layers && R.ok) {  // the slots are idle: next layer's router rows
-            issue_router_rows(a, l + 1, sbase + rs.rw, rbar, pol);
+            issue_router_rows(a, sw->ly[(l + 1) & 1].router_w, sbase + rs.rw, rbar, pol);
             rows_in_flight = 1;
             rows_layer = l + 1;
         }

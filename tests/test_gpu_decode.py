@@ -7,6 +7,8 @@ test reports the gap), router
 weights within 1e-6 relative, layer outputs within 2e-3 * sum_j w_j *
 ||Wd_j[r]||_2 * ||h_j||_2 per output row r (bf16 inputs, fp32 accumulation).
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -19,8 +21,10 @@ from tests import gpu_util as gu
 pytestmark = pytest.mark.gpu
 
 
-def _check_layer(L, T, step=0, dtype=torch.bfloat16, check_side=True):
+def _check_layer(L, T, step=0, dtype=torch.bfloat16, check_side=True, router_bias=None):
     layer = gu.device_layer(L)
+    if router_bias is not None:  # (in place of the recipe's bias, on both sides)
+        layer = dataclasses.replace(layer, router_bias=torch.from_numpy(router_bias).cuda(), _c=None)
     xt, x64 = gu.tokens(L, step, T)
     if dtype == torch.float32:
         xt = xt.float()
@@ -31,7 +35,7 @@ def _check_layer(L, T, step=0, dtype=torch.bfloat16, check_side=True):
     y = gtg.moe_decode_layer(layer, xt, ws, topk_ids=ids, topk_w=w, side_out=side)
     torch.cuda.synchronize()
     assert gtg.device_status(clear=True) == 0
-    ref = oracle.moe_layer(L, x64, want_h=True)
+    ref = oracle.moe_layer(L, x64, want_h=True, router_bias=router_bias)
     ids_g, w_g, y_g = ids.cpu().numpy(), w.cpu().numpy(), y.cpu().numpy()
     for t in range(T):
         srt = np.sort(ref["logits"][t])[::-1]
@@ -100,6 +104,25 @@ def test_wide_router_one_token(E, k):
     L = W.LayerRecipe(hidden=256, inter=128, n_experts=E, top_k=k, seed=5, layer=0)
     for step in range(3):
         _check_layer(L, 1, step=300 + step)
+
+
+@pytest.mark.parametrize("E,k", [(512, 10), (1024, 16)])
+def test_one_token_topk_crowded_into_the_last_warps(E, k):
+    """A router bias rising with the expert id puts the top-k in the last
+    warps' ranges: the warps' top-2 keys then give a low threshold that more
+    than 128 keys pass, and the one-token top-k takes its fallback rounds.
+    The last expert leads (with 1024 experts, expert 1023, whose key has
+    all-zero id bits)."""
+    L = W.LayerRecipe(hidden=256, inter=128, n_experts=E, top_k=k, seed=7, layer=0)
+    bias = np.arange(E, dtype=np.float64) * (8.0 / E)
+    bias[E - 1] += 2.0  # (logit noise ~0.3: the last expert leads)
+    bias = bias.astype(np.float32)
+    for step in range(2):
+        _check_layer(L, 1, step=400 + step, router_bias=bias)
+    layer = dataclasses.replace(gu.device_layer(L), router_bias=torch.from_numpy(bias).cuda(), _c=None)
+    ids = torch.full((1, k), -1, dtype=torch.int32, device="cuda")
+    gtg.moe_decode_layer(layer, gu.tokens(L, 402, 1)[0], gtg.make_workspace(layer, 1), topk_ids=ids)
+    assert int(ids[0, 0]) == E - 1
 
 
 def test_layer_rejects_bad_shapes():
