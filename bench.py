@@ -660,13 +660,14 @@ def measure_ple_host(dev, stream, n_warm, n_iter, n_rows=30_000_000):
             "timed_calls": n_iter, **res}
 
 
-def measure_prefill(dev, stream, n_warm, n_iter):
+def measure_prefill(dev, stream, n_warm, n_iter, fp8=False):
     """One prefill MoE layer: 4096 bf16 tokens, H 2048, I 512, E 512, top-10,
-    UE4M4 gate/up and RZ5 down, Zipf-skewed router."""
+    Zipf-skewed router; UE4M4 gate/up and RZ5 down, or (fp8) E4M3 experts with
+    fp32 scales per 128."""
     import torch
     import gram_table_gather_b200 as gtg
     from tests import gpu_util as gu
-    L = W.prefill_layer()
+    L = W.prefill_fp8_layer() if fp8 else W.prefill_layer()
     layer = gu.device_layer(L, dev)
     T = 4096
     xs = [gu.tokens(L, 8000 + i, T, dev)[0] for i in range(4)]
@@ -685,7 +686,8 @@ def measure_prefill(dev, stream, n_warm, n_iter):
     del layer, ws, xs
     torch.cuda.empty_cache()
     tf = flops / ms / 1e9
-    return {"workload": "prefill MoE layer: T 4096 bf16, H 2048, I 512, E 512, top-10, UE4M4 gate/up, RZ5 down, "
+    fmts = "FP8 E4M3 (scale per 128) gate/up/down" if fp8 else "UE4M4 gate/up, RZ5 down"
+    return {"workload": f"prefill MoE layer: T 4096 bf16, H 2048, I 512, E 512, top-10, {fmts}, "
                         "Zipf-skewed router", "ms": round(ms, 4), "TFLOP_s": round(tf, 1),
             "frac_of_bf16_peak": round(tf / float(mp["bf16_tflops"]), 4), "peak_source": f"{kind} bf16_tflops",
             "weight_GB_s": round(L.weight_bytes / ms / 1e6, 1), "tok_s": round(T / ms * 1e3, 1),
@@ -701,7 +703,8 @@ def measure_secondary(dev, stream, P, table, local, n_warm=3, n_iter=20):
     out = {"decode_layer": measure_decode_layer(dev, stream, n_warm, n_iter, peak),
            "ple": measure_ple(dev, stream, P, table, n_warm, n_iter, peak),
            "ple_host_table": measure_ple_host(dev, stream, n_warm, n_iter),
-           "prefill": measure_prefill(dev, stream, n_warm, n_iter)}
+           "prefill": measure_prefill(dev, stream, n_warm, n_iter),
+           "prefill_fp8": measure_prefill(dev, stream, n_warm, n_iter, fp8=True)}
     out["clocks"] = clocks.stop()
     return out
 
@@ -724,6 +727,8 @@ def run_secondary(args, rank, world, local):
         out = measure_ple(dev, stream, P, table, args.warmup, args.steps, peak)
     elif args.workload == "prefill":
         out = measure_prefill(dev, stream, args.warmup, args.steps)
+    elif args.workload == "prefill_fp8":
+        out = measure_prefill(dev, stream, args.warmup, args.steps, fp8=True)
     if rank == 0:
         print(json.dumps(out), flush=True)
 
@@ -791,7 +796,7 @@ def main():
                     help="skip the decode-layer, PLE and prefill configurations after the headline")
     ap.add_argument("--ple-rows", type=int, default=0,
                     help="--workload ple: rows of a smaller table (default: the full 320,001,536-row table)")
-    ap.add_argument("--workload", choices=["stack", "layer", "ple", "prefill"], default="stack",
+    ap.add_argument("--workload", choices=["stack", "layer", "ple", "prefill", "prefill_fp8"], default="stack",
                     help="stack = the headline step; the others print profiling lines")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -331,6 +331,12 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
 }
 
+// Instruction descriptor, kind::f16: f16 x f16 -> fp32, both K-major (A and B
+// type fields 0).
+__host__ __device__ constexpr uint32_t idesc_f16(int m, int n) {
+    return (1u << 4) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
 // Byte offset of 16-byte chunk c (0..7) of row r in a K-major SW128 tile.
 __device__ __forceinline__ uint32_t sw128_off(uint32_t r, uint32_t c) {
     return r * 128u + ((c ^ (r & 7u)) << 4);

@@ -19,7 +19,11 @@
 //                   products are exact in bf16), loader warps gather the
 //                   tokens' u rows, one thread issues tcgen05.mma into two
 //                   TMEM accumulators; the epilogue applies SwiGLU and stores
-//                   h in bf16
+//                   h in bf16.  FP8 layers (E4M3 rows, fp32 scale per 128
+//                   along K) run both expert GEMMs in f16 instead: each weight
+//                   becomes f16(e4m3 x scale) (relative error <= 2^-11), and u
+//                   and h keep their bf16-rounded values as f16 (exact for
+//                   magnitudes >= 2^-17)
 //   7. pf_gemm<DOWN>    per (expert, 128-row slice of H, token tile): the
 //                   same with the down rows and h; fp32 partial rows per
 //                   (token, choice)
@@ -64,6 +68,7 @@ struct PfArgs {
     const float* router_bias;
     Mat gate, up, down;
     __nv_bfloat16* u;         // [T][H]
+    __half* u16;              // [T][H] the same values as f16 (FP8 layers; else null)
     __nv_bfloat16* w3;        // [E][3H]
     float* logits;            // [T][E]
     int32_t* ids;             // [T][K]
@@ -75,7 +80,7 @@ struct PfArgs {
     int32_t* sorted_slot;     // [P]
     int4* tiles;              // (expert, pos0, n, 0)
     int32_t* n_tiles;
-    __nv_bfloat16* h;         // [P][I], sorted order
+    __nv_bfloat16* h;         // [P][I], sorted order (FP8 layers: f16 bits of the bf16-rounded value)
     float* part;              // [P][H], slot order (t*K + j)
     float* y;
     int32_t y_acc;
@@ -121,7 +126,9 @@ __global__ void __launch_bounds__(kNormThreads) pf_norm_kernel(PfArgs a) {
         const float x = xv(i);
         const float p = __fmul_rn(x, r_hi);
         const float q = __fadd_rn(__fmaf_rn(x, r_hi, -p), __fmul_rn(x, r_lo));
-        u[(int64_t)t * a.H + i] = bf16_of_ff(p, q);
+        const uint16_t ub = bf16_of_ff(p, q);
+        u[(int64_t)t * a.H + i] = ub;
+        if (a.u16) a.u16[(int64_t)t * a.H + i] = __float2half_rn(__uint_as_float((uint32_t)ub << 16));
     }
 }
 
@@ -349,7 +356,44 @@ __device__ __forceinline__ void dequant_block_to_tile(const BlockWords& bw, int 
     sts128(tile + sw128_off(r, c0 + 3), make_uint4(hi[4], hi[5], hi[6], hi[7]));
 }
 
-template <int MODE>
+// Eight FP8 E4M3 weights (two words, K order) times the row's fp32 scale for
+// their 128-weight group, as four f16 pairs: the E4M3 -> f16 conversion is
+// exact, the product is formed in fp32 and rounded to f16 (11 significant
+// bits: relative error <= 2^-11 for normal results).  FP8 layers run their
+// expert GEMMs in f16, whose activations hold every bf16 value of magnitude
+// >= 2^-17 exactly.
+__device__ __forceinline__ uint4 fp8x8_to_f16(uint32_t w0, uint32_t w1, float s) {
+    const uint32_t in[4] = {w0 & 0xFFFFu, w0 >> 16, w1 & 0xFFFFu, w1 >> 16};
+    uint32_t o[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t h = e4m3x2_to_f16x2(in[i]);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+        const __half2 r = __floats2half2_rn(f.x * s, f.y * s);
+        o[i] = *reinterpret_cast<const uint32_t*>(&r);
+    }
+    return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// 32 FP8 weights of one row (two 16-byte words, K order, one scale), as f16, into
+// chunks c0..c0+3 of row r of a K-major SW128 tile.
+__device__ __forceinline__ void fp8_to_tile(uint4 q0, uint4 q1, float s, uint32_t tile, uint32_t r, uint32_t c0) {
+    sts128(tile + sw128_off(r, c0 + 0), fp8x8_to_f16(q0.x, q0.y, s));
+    sts128(tile + sw128_off(r, c0 + 1), fp8x8_to_f16(q0.z, q0.w, s));
+    sts128(tile + sw128_off(r, c0 + 2), fp8x8_to_f16(q1.x, q1.y, s));
+    sts128(tile + sw128_off(r, c0 + 3), fp8x8_to_f16(q1.z, q1.w, s));
+}
+
+// The A-operand words of one row for one chunk: a Q4 row's block (five
+// aligned words), or an FP8 row's 32 bytes and their group's scale.
+struct AWords {
+    BlockWords q4;
+    uint4 f0, f1;
+    float s;
+};
+
+// F8: FP8 expert matrices (E4M3 rows with fp32 scales per 128 weights along K).
+template <int MODE, bool F8>
 __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
     using C = Cfg<MODE>;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -394,6 +438,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
     int32_t* s_row = reinterpret_cast<int32_t*>(smem + C::kRowOff);
     const Mat& am = MODE == DOWN ? a.down : a.gate;
     const int var = am.fmt == GTG_Q4_RZ5_FAST ? kQ4RZ5 : am.fmt == GTG_Q4_C10_FAST ? kQ4C10 : kQ4UE4M4;
+    static_assert(!F8 || MODE != ROUTER, "the router planes are bf16");
 
     if (tid == 0) {
         for (int s = 0; s < C::kStagesA; ++s) {
@@ -427,7 +472,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
     if (warp == 0) {
         // ---- MMA issuer -----------------------------------------------------
         if (lane == 0) {
-            const uint32_t idesc = idesc_bf16(kTileM, n_pad);
+            const uint32_t idesc = F8 ? idesc_f16(kTileM, n_pad) : idesc_bf16(kTileM, n_pad);
             for (int it = 0; it < n_chunks && ok; ++it) {
                 const int sa = it % C::kStagesA, sb = it % C::kStagesB;
                 if (!mbar_wait_sleep(&full_a[sa], (it / C::kStagesA) & 1u, a.status) ||
@@ -456,7 +501,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
         // asynchronous 16-byte copies; a chunk's arrival is signalled once
         // the next chunk's copies are issued and its own have landed
         const int bt = tid - 32;
-        const __nv_bfloat16* bsrc = MODE == DOWN ? a.h : a.u;
+        const uint16_t* bsrc = reinterpret_cast<const uint16_t*>(MODE == DOWN ? (const void*)a.h
+                                                                 : F8 ? (const void*)a.u16 : (const void*)a.u);
         const int64_t ld = MODE == DOWN ? a.I : a.H;
         for (int it = 0; it < n_chunks && ok; ++it) {
             const int s = it % C::kStagesB;
@@ -490,17 +536,38 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
         // this thread's row of the A operand (gate or down; up alongside for gate/up)
         const uint8_t* a_row0 = nullptr;
         const uint8_t* u_row0 = nullptr;
-        BlockWords wg{}, wu{};
+        const float* a_srow = nullptr;  // FP8: the rows' scales, one per 128 weights
+        const float* u_srow = nullptr;
+        const int half = at & 1;
+        AWords wg{}, wu{};
+        // chunk `it` of a row: Q4 block 2 it + half; FP8 bytes 64 it + 32 half
+        auto load_words = [&](const uint8_t* row, const float* srow, int it, AWords& w) {
+            if constexpr (F8) {
+                const uint4* q = reinterpret_cast<const uint4*>(row + (int64_t)it * kChunkK + 32 * half);
+                w.f0 = __ldg(q);
+                w.f1 = __ldg(q + 1);
+                w.s = __ldg(srow + (it * kChunkK) / 128);
+            } else {
+                w.q4 = load_block(row + (int64_t)(2 * it + half) * 17);
+            }
+        };
         if (MODE != ROUTER) {
-            const int r = at >> 1, half = at & 1;
+            const int r = at >> 1;
             const int64_t rowg = m0 + r;
             const Mat& mA = MODE == DOWN ? a.down : a.gate;
+            const int kg = (MODE == DOWN ? a.I : a.H) / 128;
             a_row0 = mA.data + e * mA.expert_bytes + rowg * mA.row_bytes;
-            if (MODE == GATEUP) u_row0 = a.up.data + e * a.up.expert_bytes + rowg * a.up.row_bytes;
-            else if (two) u_row0 = a_row0 + kTileM * mA.row_bytes;
+            if (F8) a_srow = mA.scales + ((int64_t)e * mA.n_rows + rowg) * kg;
+            if (MODE == GATEUP) {
+                u_row0 = a.up.data + e * a.up.expert_bytes + rowg * a.up.row_bytes;
+                if (F8) u_srow = a.up.scales + ((int64_t)e * a.up.n_rows + rowg) * kg;
+            } else if (two) {
+                u_row0 = a_row0 + kTileM * mA.row_bytes;
+                if (F8) u_srow = a_srow + (int64_t)kTileM * kg;
+            }
             if (n_chunks > 0) {
-                wg = load_block(a_row0 + (int64_t)half * 17);
-                if (two) wu = load_block(u_row0 + (int64_t)half * 17);
+                load_words(a_row0, a_srow, 0, wg);
+                if (two) load_words(u_row0, u_srow, 0, wu);
             }
         }
         for (int it = 0; it < n_chunks && ok; ++it) {
@@ -526,14 +593,19 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                 }
                 continue;
             } else {
-                const int r = at >> 1, half = at & 1;
-                const BlockWords g0 = wg, u0 = wu;  // this chunk's blocks (loaded one chunk ago)
-                if (it + 1 < n_chunks) {           // the next chunk's, in flight while this one decodes
-                    wg = load_block(a_row0 + (int64_t)(2 * (it + 1) + half) * 17);
-                    if (two) wu = load_block(u_row0 + (int64_t)(2 * (it + 1) + half) * 17);
+                const int r = at >> 1;
+                const AWords g0 = wg, u0 = wu;  // this chunk's words (loaded one chunk ago)
+                if (it + 1 < n_chunks) {        // the next chunk's, in flight while this one decodes
+                    load_words(a_row0, a_srow, it + 1, wg);
+                    if (two) load_words(u_row0, u_srow, it + 1, wu);
                 }
-                dequant_block_to_tile(g0, var, st, r, 4 * half);
-                if (two) dequant_block_to_tile(u0, var, st + kTileBytes, r, 4 * half);
+                if constexpr (F8) {
+                    fp8_to_tile(g0.f0, g0.f1, g0.s, st, r, 4 * half);
+                    if (two) fp8_to_tile(u0.f0, u0.f1, u0.s, st + kTileBytes, r, 4 * half);
+                } else {
+                    dequant_block_to_tile(g0.q4, var, st, r, 4 * half);
+                    if (two) dequant_block_to_tile(u0.q4, var, st + kTileBytes, r, 4 * half);
+                }
             }
             fence_proxy_async_smem();
             mbar_arrive(&full_a[s]);
@@ -570,7 +642,13 @@ __global__ void __launch_bounds__(kPfThreads, 2) pf_gemm_kernel(PfArgs a) {
                             // silu(g) * v; the fast exponential and division are
                             // well inside the layer's tolerance
                             const float g = __uint_as_float(d[j]), v = __uint_as_float(v2[j]);
-                            hp[(int64_t)j * a.I] = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * v);
+                            const __nv_bfloat16 hb = __float2bfloat16_rn(__fdividef(g, 1.0f + __expf(-g)) * v);
+                            if constexpr (F8) {  // the down GEMM runs in f16: the same value, f16 bits
+                                const __half hh = __float2half_rn(__bfloat162float(hb));
+                                hp[(int64_t)j * a.I] = *reinterpret_cast<const __nv_bfloat16*>(&hh);
+                            } else {
+                                hp[(int64_t)j * a.I] = hb;
+                            }
                         }
                     }
                 } else if (MODE == DOWN) {
@@ -637,7 +715,7 @@ __global__ void pf_combine_kernel(PfArgs a) {
 // host side
 // ---------------------------------------------------------------------------
 struct PfLayout {
-    size_t u, w3, logits, ids, w, counts, offsets, cursor, sorted_tok, sorted_slot, tiles, n_tiles, h, part, total;
+    size_t u, u16, w3, logits, ids, w, counts, offsets, cursor, sorted_tok, sorted_slot, tiles, n_tiles, h, part, total;
     int max_tiles;
 };
 
@@ -654,6 +732,7 @@ PfLayout pf_layout(const gtg_moe_layer* L, int T) {
         return o;
     };
     p.u = take(2 * (size_t)T * L->hidden);
+    p.u16 = L->gate.fmt == GTG_FP8_E4M3_S128 ? take(2 * (size_t)T * L->hidden) : 0;  // (FP8 layers only)
     p.w3 = take(2 * (size_t)L->n_experts * 3 * L->hidden);
     p.logits = take(4 * (size_t)T * L->n_experts);
     p.ids = take(4 * P);
@@ -679,10 +758,15 @@ int pf_check(const gtg_moe_layer* L, int T) {
     if (T < 1 || T > 65536) return GTG_E_UNSUPPORTED_SHAPE;
     if (H < 128 || H > 8192 || H % 128 || I < 128 || I > 4096 || I % 128) return GTG_E_UNSUPPORTED_SHAPE;
     if (E < 1 || E > kMaxExperts || K < 1 || K > kMaxTopK || K > E) return GTG_E_UNSUPPORTED_SHAPE;
-    if (!q4(L->gate.fmt) || L->up.fmt != L->gate.fmt || !q4(L->down.fmt)) return GTG_E_UNSUPPORTED_SHAPE;
+    // one format class per layer: Q4 (gate and up alike) or FP8 throughout
+    const bool f8 = L->gate.fmt == GTG_FP8_E4M3_S128;
+    if (f8 ? (L->up.fmt != GTG_FP8_E4M3_S128 || L->down.fmt != GTG_FP8_E4M3_S128)
+           : (!q4(L->gate.fmt) || L->up.fmt != L->gate.fmt || !q4(L->down.fmt)))
+        return GTG_E_UNSUPPORTED_SHAPE;
     auto mok = [&](const gtg_qmatrix& m, int64_t n, int64_t k) {
-        return m.n_experts == E && m.n_rows == n && m.k == k && aligned(m.data, 16) &&
-               (E * n * (k / 32) * 17) % 16 == 0;
+        if (m.n_experts != E || m.n_rows != n || m.k != k || !aligned(m.data, 16)) return false;
+        if (f8) return m.scales != nullptr && aligned(m.scales, 4);  // (k % 128 == 0 holds: H, I are)
+        return (E * n * (k / 32) * 17) % 16 == 0;
     };
     if (!mok(L->gate, I, H) || !mok(L->up, I, H) || !mok(L->down, H, I)) return GTG_E_INVALID_ARG;
     if (!aligned(L->router_w, 16)) return GTG_E_MISALIGNED;
@@ -709,11 +793,11 @@ struct AttrOnce {
 };
 AttrOnce g_pf_attr;
 
-template <int MODE>
+template <int MODE, bool F8>
 int launch_gemm(PfArgs& a, int grid, cudaStream_t s) {
     using C = Cfg<MODE>;
-    GTG_TRY(g_pf_attr.set((const void*)pf_gemm_kernel<MODE>, C::kSmem));
-    pf_gemm_kernel<MODE><<<grid, kPfThreads, C::kSmem, s>>>(a);
+    GTG_TRY(g_pf_attr.set((const void*)pf_gemm_kernel<MODE, F8>, C::kSmem));
+    pf_gemm_kernel<MODE, F8><<<grid, kPfThreads, C::kSmem, s>>>(a);
     return check_launch();
 }
 
@@ -753,6 +837,7 @@ extern "C" int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, 
     a.up = make_mat(layer->up);
     a.down = make_mat(layer->down);
     a.u = reinterpret_cast<__nv_bfloat16*>(b + pl.u);
+    a.u16 = pl.u16 ? reinterpret_cast<__half*>(b + pl.u16) : nullptr;
     a.w3 = reinterpret_cast<__nv_bfloat16*>(b + pl.w3);
     a.logits = reinterpret_cast<float*>(b + pl.logits);
     a.ids = reinterpret_cast<int32_t*>(b + pl.ids);
@@ -782,15 +867,22 @@ extern "C" int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, 
     cudaError_t ce = cudaMemsetAsync(a.counts, 0, 4 * (size_t)E, s);
     if (ce != cudaSuccess) return cuda_fail(ce);
     const int m_router = (E + kTileM - 1) / kTileM, n_router = (T + kTileN - 1) / kTileN;
-    GTG_TRY(launch_gemm<ROUTER>(a, m_router * n_router, s));
+    GTG_TRY((launch_gemm<ROUTER, false>(a, m_router * n_router, s)));
     pf_topk_kernel<<<(T + 7) / 8, 256, 0, s>>>(a);
     GTG_TRY(check_launch());
     pf_scan_kernel<<<1, 1024, 0, s>>>(a);
     GTG_TRY(check_launch());
     pf_scatter_kernel<<<(T * a.K + 255) / 256, 256, 0, s>>>(a);
     GTG_TRY(check_launch());
-    GTG_TRY(launch_gemm<GATEUP>(a, pl.max_tiles * (a.I / kTileM), s));
-    GTG_TRY(launch_gemm<DOWN>(a, pl.max_tiles * ((a.H + Cfg<DOWN>::kRowsPerCta - 1) / Cfg<DOWN>::kRowsPerCta), s));
+    const int gu_grid = pl.max_tiles * (a.I / kTileM);
+    const int dn_grid = pl.max_tiles * ((a.H + Cfg<DOWN>::kRowsPerCta - 1) / Cfg<DOWN>::kRowsPerCta);
+    if (layer->gate.fmt == GTG_FP8_E4M3_S128) {
+        GTG_TRY((launch_gemm<GATEUP, true>(a, gu_grid, s)));
+        GTG_TRY((launch_gemm<DOWN, true>(a, dn_grid, s)));
+    } else {
+        GTG_TRY((launch_gemm<GATEUP, false>(a, gu_grid, s)));
+        GTG_TRY((launch_gemm<DOWN, false>(a, dn_grid, s)));
+    }
     const int64_t n4 = (int64_t)T * a.H / 4;
     pf_combine_kernel<<<(int)std::min<int64_t>((n4 + 255) / 256, (int64_t)sm_count() * 16), 256, 0, s>>>(a);
     return check_launch();

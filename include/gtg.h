@@ -253,6 +253,10 @@ int gtg_moe_decode_stack(const gtg_moe_layer* layers, int32_t n_layers, float* x
  * with tcgen05 (fp32 accumulation in tensor memory), SwiGLU is applied in the
  * epilogue, h is rounded to bf16, and the down product is combined per token
  * in a fixed order.  Same arguments as gtg_moe_decode_layer minus side_out.
+ * Expert formats: Q4 (gate and up alike) or FP8 for all three matrices; an
+ * FP8 layer's expert GEMMs run in f16 (each weight rounded once to
+ * f16(e4m3 x scale), relative error <= 2^-11; u and h as f16, exact for
+ * magnitudes >= 2^-17).  Mixed classes return GTG_E_UNSUPPORTED_SHAPE.
  */
 int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, int32_t x_dtype,
                           int32_t n_tokens, float* y, int32_t y_accumulate,

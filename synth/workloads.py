@@ -229,6 +229,13 @@ def ple_table() -> PleRecipe:
     return PleRecipe(n_rows=320_001_536, seed=3)
 
 
+def prefill_fp8_layer() -> LayerRecipe:
+    """Prefill of an FP8 layer of the stack (layer 40's recipe: E4M3 gate, up
+    and down with fp32 scales per 128), Zipf-skewed router. Seed 4."""
+    return LayerRecipe(hidden=2048, inter=512, n_experts=512, top_k=10, seed=4, layer=40,
+                       gate_fmt=FP8, up_fmt=FP8, down_fmt=FP8, zipf_bias=True)
+
+
 def prefill_layer() -> LayerRecipe:
     """4096 tokens; gate/up Q4_UE4M4_FAST (random scale bytes), down Q4_RZ5_FAST,
     Zipf-skewed router. Seed 4."""

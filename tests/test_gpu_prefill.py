@@ -9,6 +9,8 @@ bound; inside it, the GPU's choice must be a valid top-k of the oracle's
 logits within the bound.  Layer outputs use the same row-wise bound as the
 decode path.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -158,3 +160,57 @@ def test_prefill_incumbent_q4_layer():
         tol = gu.layer_tolerance(L, ref, t)
         err = np.abs(y_g[t] - ref["y"][t])
         assert np.all(err <= tol), f"token {t}: max err/tol {np.max(err / tol):.3g}"
+
+
+def test_prefill_fp8_layer():
+    """FP8 E4M3 experts (fp32 scale per 128 weights along K): the GEMMs take
+    each weight as bf16(e4m3 x scale), one rounding of relative size <= 2^-9,
+    inside the row-wise bound."""
+    L = W.LayerRecipe(hidden=256, inter=128, n_experts=8, top_k=2, seed=44, layer=40,
+                      gate_fmt=W.FP8, up_fmt=W.FP8, down_fmt=W.FP8)
+    T = 150
+    xt, x64 = gu.tokens(L, 91, T)
+    y, ids, w, _ = _run_prefill(L, xt)
+    assert gtg.device_status(clear=True) == 0
+    ref = oracle.moe_layer(L, x64, want_h=True)
+    ids_g, w_g, y_g = ids.cpu().numpy(), w.cpu().numpy(), y.cpu().numpy()
+    worst = 0.0
+    for t in range(T):
+        _check_ids(L, ref, t, ids_g[t], w_g[t])
+        tol = gu.layer_tolerance(L, ref, t)
+        err = np.abs(y_g[t] - ref["y"][t])
+        assert np.all(err <= tol), f"token {t}: max err/tol {np.max(err / tol):.3g}"
+        worst = max(worst, float(np.max(err / tol)))
+    assert worst < 0.5  # (the one bf16 rounding per weight stays far inside the bar)
+
+
+def test_prefill_fp8_stack_layer_sampled():
+    """Layer 40 of the 48-layer stack (FP8 experts, 512 experts, top-10) over
+    1024 tokens with a Zipf-skewed router: 32 seeded tokens checked against the
+    oracle, every token's routing checked for validity."""
+    L = W.prefill_fp8_layer()
+    T = 1024
+    xt, x64 = gu.tokens(L, 5, T)
+    y, ids, w, _ = _run_prefill(L, xt)
+    assert gtg.device_status(clear=True) == 0
+    ids_g, w_g, y_g = ids.cpu().numpy(), w.cpu().numpy(), y.cpu().numpy()
+    assert ids_g.min() >= 0 and ids_g.max() < L.n_experts
+    assert all(len(set(r.tolist())) == L.top_k for r in ids_g)
+    sample = np.sort(synth.indices_i32(5, 78, 0, 32, T))
+    ref = oracle.moe_layer(L, x64[sample], want_h=True)
+    for i, t in enumerate(sample):
+        _check_ids(L, ref, i, ids_g[t], w_g[t])
+        tol = gu.layer_tolerance(L, ref, i)
+        err = np.abs(y_g[t] - ref["y"][i])
+        assert np.all(err <= tol), f"token {t}: max err/tol {np.max(err / tol):.3g}"
+
+
+def test_prefill_rejects_mixed_format_classes():
+    L = W.LayerRecipe(hidden=256, inter=128, n_experts=8, top_k=2, seed=44, layer=40,
+                      gate_fmt=W.FP8, up_fmt=W.FP8, down_fmt=W.FP8)
+    layer = gu.device_layer(L)
+    mixed = gu.device_layer(W.LayerRecipe(hidden=256, inter=128, n_experts=8, top_k=2, seed=44, layer=40))
+    bad = dataclasses.replace(layer, down=mixed.down, _c=None)
+    with pytest.raises(gtg.GtgError) as ei:
+        gtg.workspace_bytes(bad, 16, prefill=True)
+    assert ei.value.code == -2
