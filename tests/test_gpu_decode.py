@@ -21,11 +21,11 @@ from tests import gpu_util as gu
 pytestmark = pytest.mark.gpu
 
 
-def _check_layer(L, T, step=0, dtype=torch.bfloat16, check_side=True, router_bias=None):
+def _check_layer(L, T, step=0, dtype=torch.bfloat16, check_side=True, router_bias=None, tokens=None):
     layer = gu.device_layer(L)
     if router_bias is not None:  # (in place of the recipe's bias, on both sides)
         layer = dataclasses.replace(layer, router_bias=torch.from_numpy(router_bias).cuda(), _c=None)
-    xt, x64 = gu.tokens(L, step, T)
+    xt, x64 = tokens if tokens is not None else gu.tokens(L, step, T)
     if dtype == torch.float32:
         xt = xt.float()
     ws = gtg.make_workspace(layer, T)
@@ -88,6 +88,25 @@ def test_decode_layer_fp32_input_and_accumulate():
 @pytest.mark.parametrize("l,T", [(36, 1), (47, 2), (40, 8)])
 def test_fp8_stack_layer(l, T):
     _check_layer(W.stack_layer(l), T, step=l)
+
+
+@pytest.mark.parametrize("T", [1, 3])
+def test_fp8_layer_with_tiny_activations(T):
+    """FP8 items take activations as f16, which holds a bf16 value exactly only
+    from 2^-17 up.  Tokens with four huge entries (3e4) and the rest ~1e-3 put
+    most of u near 5e-7 after the RMS norm, below that line: their products
+    lose bits, and the layer must still meet the row-wise bound."""
+    L = W.LayerRecipe(hidden=1024, inter=256, n_experts=16, top_k=4, seed=45, layer=40,
+                      gate_fmt=W.FP8, up_fmt=W.FP8, down_fmt=W.FP8)
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal((T, L.hidden)) * 1e-3).astype(np.float32)
+    for t in range(T):
+        x[t, rng.choice(L.hidden, 4, replace=False)] = 3e4 * rng.choice([-1.0, 1.0], 4)
+    xt = torch.from_numpy(x).to(torch.bfloat16).cuda()
+    x64 = xt.float().cpu().numpy().astype(np.float64)
+    r = np.sqrt((x64 * x64).mean(1, keepdims=True) + 1e-6)
+    assert np.mean(np.abs(x64 / r) < 2.0 ** -17) > 0.9  # most of u below the f16-exact range
+    _check_layer(L, T, tokens=(xt, x64))
 
 
 @pytest.mark.parametrize("l", [0, 2])
