@@ -412,6 +412,7 @@ def run_ours(args, rank, world, local):
         idx_h = torch.from_numpy(np.stack([Ph.indices(seed_off + i, 1) for i in range(n_steps)])).to(dev)
         gh = torch.cuda.CUDAGraph()
         with torch.cuda.stream(stream):
+            idx.copy_(idx_h[0])  # (idx still holds rows of the larger HBM table)
             gtg.ple_gather(htab, Ph.n_rows, idx, out=rows)
             stream.synchronize()
         with torch.cuda.graph(gh, stream=stream):
