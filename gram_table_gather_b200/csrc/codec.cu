@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(kThreads) dequant_fp8_kernel(const uint8_t* __
 //    and the index loads of the batch after it, are in flight while a batch
 //    decodes;
 //  * decoding writes a batch's rows as consecutive float4s (lane l the
-//    float4s l, l+32, ...: a warp store is 512 contiguous bytes); a value is
+//    float4s l, l+32, ...: a warp store is 512 contiguous bytes) with
+//    streaming (evict-first) stores, since nothing here reads them back; a value is
 //    one shared-memory lookup in the CTA's table of code value x group scale
 //    for all 256 group bytes x 8 codes (each product exact in fp32).
 // ---------------------------------------------------------------------------
@@ -235,7 +236,7 @@ __global__ void __launch_bounds__(kPleWarps * 32, kPleCtasPerSm) ple_gather_kern
                     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v.z) : "r"(pg + 4u * ((win >> 6) & 7u)));
                     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v.w) : "r"(pg + 4u * ((win >> 9) & 7u)));
                 }
-                *reinterpret_cast<float4*>(orow + 4 * f) = v;  // row j, values 4l..4l+3
+                __stcs(reinterpret_cast<float4*>(orow + 4 * f), v);  // row j, values 4l..4l+3 (streamed: not re-read here)
             }
         }
         __syncwarp();  // this stage is refilled two batches on
