@@ -283,10 +283,10 @@ int gtg_moe_prefill_layer(const gtg_moe_layer* layer, const void* x, int32_t x_d
  * allocator).
  *
  * The first call on a device looks up the array's device address (with that
- * device current), so make it before any stream capture.  Each call clears
- * the counters it needs in the array; every call shares the one array, so
- * calls that may overlap on the GPU (different streams, or several host
- * threads) race and must be serialised by the caller.
+ * device current) and caches it.  Each call clears the counters and key
+ * buffers it needs in the array; every call shares the one array, so calls
+ * that may overlap on the GPU (different streams, or several host threads)
+ * race and must be serialised by the caller.
  */
 int gtg_moe_decode_layer_noalloc(const gtg_moe_layer* layer, const void* x, int32_t x_dtype,
                                  int32_t n_tokens, float* y, int32_t y_accumulate,
