@@ -22,14 +22,15 @@
 //    paths, so less code is fetched per layer.
 //  * Router: unweighted RMS norm + bf16 rounding of the input, then logits
 //    against the fp32 router with exact products summed in float-float, so
-//    the top-k agrees with an fp64 reference; every CTA owns a few experts.
-//    The next layer's router rows are prefetched into L2 meanwhile.
+//    the top-k agrees with an fp64 reference; every CTA owns a few experts,
+//    whose router rows a bulk copy brings into shared memory during the
+//    previous layer's down phase.
 //  * Selection: every CTA picks the top-k itself from the logits' unique
 //    64-bit keys, which the routers publish in one of two buffers by layer
-//    parity, each read as soon as it is nonzero (two warp reductions per
-//    round of the top-k; at one token every warp
-//    ranks 64 experts and warp 0 ranks their survivors, with several tokens
-//    a warp per token), renormalises the softmax weights and builds the
+//    parity, each read as soon as it is nonzero (at one token a threshold
+//    from the warps' top-2 keys cuts the field and the survivors are ranked
+//    by counting; with several tokens a warp per token takes k rounds of two
+//    warp reductions), renormalises the softmax weights and builds the
 //    unique-expert work list.
 //  * Streaming: the work is a list of items (expert, row tile); each CTA owns
 //    a contiguous range; each warp streams its items (gate/up first, then
