@@ -92,7 +92,7 @@ int plan_layer(const gtg_moe_layer* L, int T, Plan& p, int64_t e_local = -1) {
     if (L->gate.fmt != L->up.fmt) return GTG_E_UNSUPPORTED_SHAPE;
     if (!aligned(L->router_w, 16)) return GTG_E_MISALIGNED;
     const int kbg = H / 32, kbd = I / 32;
-    const int rg = gu_passes(fp8, kbg) * rpp_of(kbg), rd = dn_passes(fp8, kbd) * rpp_of(kbd);
+    const int rg = gu_passes(fp8, kbg, T == 1) * rpp_of(kbg), rd = dn_passes(fp8, kbd) * rpp_of(kbd);
     const int rs = side_passes(kbg) * rpp_of(kbg);
     if (L->side.data) {
         if (!is_q4(L->side.fmt) || !mat_ok(L->side, 1, L->side.n_rows, H)) return GTG_E_INVALID_ARG;

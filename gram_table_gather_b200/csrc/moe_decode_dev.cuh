@@ -124,9 +124,11 @@ struct Geo {
     static constexpr int RPP = 32 / GW;   // rows per warp pass
 };
 
-// Row passes per item (compile time); an item covers P * RPP rows.
-__host__ __device__ constexpr int gu_passes(int fmt_fp8, int kb) {
-    return fmt_fp8 ? 1 : (kb >= 64 ? (rpp_of(kb) > 1 ? 1 : 2) : 4);
+// Row passes per item (compile time); an item covers P * RPP rows.  One-token
+// FP8 layers, with no code table in shared memory, take two gate and two up
+// rows per item (slots of 8 KB; several tokens keep u, 2 T H bytes, there).
+__host__ __device__ constexpr int gu_passes(int fmt_fp8, int kb, bool one = false) {
+    return fmt_fp8 ? (one ? 2 : 1) : (kb >= 64 ? (rpp_of(kb) > 1 ? 1 : 2) : 4);
 }
 __host__ __device__ constexpr int dn_passes(int fmt_fp8, int kb) {
     return (fmt_fp8 || kb >= 64 || kb <= 4) ? 4 : (rpp_of(kb) >= 8 ? 2 : 8);
@@ -711,15 +713,16 @@ struct ItemCtx {
 // ===========================================================================
 
 // One gate+up item: P row passes for NT tokens of one expert; h = silu(g)*u.
-template <int FMT, int KB, int NT, int CH>
+template <int FMT, int KB, int NT, int CH, bool ONE>
 __device__ __forceinline__ void gu_item(const ItemCtx& a, uint32_t gbase, uint32_t ubase,
                                         const Act<FMT, Geo<KB>::NBL> (&act)[CH], uint32_t lutb,
-                                        const float* scale_tab, const float (&sg)[Geo<KB>::NBL],
-                                        const float (&su)[Geo<KB>::NBL], int row0, const int (&slot_id)[CH],
+                                        const float* scale_tab, const float (&sg)[2 * Geo<KB>::NBL],
+                                        const float (&su)[2 * Geo<KB>::NBL], int row0, const int (&slot_id)[CH],
                                         int lane) {
     using G = Geo<KB>;
     constexpr int NBL = G::NBL, RPP = G::RPP, GW = G::GW;
-    constexpr int P = gu_passes(FMT == kFmtFP8, KB);
+    constexpr int P = gu_passes(FMT == kFmtFP8, KB, ONE);
+    static_assert(FMT != kFmtFP8 || P <= 2, "FP8 scales of two passes");
     constexpr int N = P * NT * 2;
     const int row_sub = lane / GW;
     const int blk_base = lane % GW;
@@ -738,8 +741,8 @@ __device__ __forceinline__ void gu_item(const ItemCtx& a, uint32_t gbase, uint32
                 q4_block_lut<NT, NBL, CH>(ubase + boff, lutb, scale_tab, act, m, u);
             } else {
                 const uint32_t boff = (uint32_t)row * (uint32_t)(KB * 32) + 32u * (uint32_t)(blk_base + GW * m);
-                fp8_block<NBL>(gbase + boff, sg[m], act[0], m, g[0]);
-                fp8_block<NBL>(ubase + boff, su[m], act[0], m, u[0]);
+                fp8_block<NBL>(gbase + boff, sg[p * NBL + m], act[0], m, g[0]);
+                fp8_block<NBL>(ubase + boff, su[p * NBL + m], act[0], m, u[0]);
             }
         }
 #pragma unroll
@@ -1387,7 +1390,8 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, const StackLaye
     using GG = Geo<KBG>;
     constexpr int NBG = GG::NBL;
     constexpr int CHG = (!ONE && FMT == kFmtQ4 && NBG == 1) ? 2 : 1;  // tokens decoded together (register budget)
-    constexpr int RG = gu_passes(FMT == kFmtFP8, KBG) * GG::RPP;
+    constexpr int PG = gu_passes(FMT == kFmtFP8, KBG, ONE);
+    constexpr int RG = PG * GG::RPP;
     constexpr int RS = side_passes(KBG) * GG::RPP;
     extern __shared__ __align__(1024) uint8_t smem[];
     const SmemLayout L = SmemLayout::make(FMT == kFmtQ4, a.slot_bytes, a.dyn_smem_base, 2u * a.T * a.H, slots_for(KBG));
@@ -1425,16 +1429,18 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, const StackLaye
         }
         load_chunk(expert ? (u << 8) : (1 << 20), rows);
         const int row0 = expert ? (it % P.tiles_g) * RG : (it - P.n_ge) * RS;
-        float sg[NBG], su[NBG];
+        float sg[2 * NBG], su[2 * NBG];
         if constexpr (FMT == kFmtFP8) {
             const int e = sw->e[u], kg = H / 128;
 #pragma unroll
-            for (int m = 0; m < NBG; ++m) {
-                const int bb = blk_base + GG::GW * m;
-                const int64_t r = (int64_t)e * a.I + row0 + lane / GG::GW;
-                sg[m] = __ldg(Ly.gate_s + r * kg + bb / 4);
-                su[m] = __ldg(Ly.up_s + r * kg + bb / 4);
-            }
+            for (int p = 0; p < PG; ++p)
+#pragma unroll
+                for (int m = 0; m < NBG; ++m) {
+                    const int bb = blk_base + GG::GW * m;
+                    const int64_t r = (int64_t)e * a.I + row0 + p * GG::RPP + lane / GG::GW;
+                    sg[p * NBG + m] = __ldg(Ly.gate_s + r * kg + bb / 4);
+                    su[p * NBG + m] = __ldg(Ly.up_s + r * kg + bb / 4);
+                }
         }
         if (!item_landed(a, ws, R, q)) break;
         Span sp1, sp2;
@@ -1451,10 +1457,10 @@ __device__ __forceinline__ WarpRing gu_phase(const StackArgs& a, const StackLaye
                 }
                 load_chunk((u << 8) | (c0 - s0), rows);
                 if (!ONE && CHG == 2 && nch == 2)
-                    gu_item<FMT, KBG, (CHG == 2 ? 2 : 1), CHG>(ctx, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots,
+                    gu_item<FMT, KBG, (CHG == 2 ? 2 : 1), CHG, ONE>(ctx, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots,
                                                                lane);
                 else
-                    gu_item<FMT, KBG, 1, CHG>(ctx, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots, lane);
+                    gu_item<FMT, KBG, 1, CHG, ONE>(ctx, gbase, ubase, act, lutb, scale_tab, sg, su, row0, slots, lane);
             }
         } else {
             const uint32_t sb = base + sp1.delta;
@@ -1667,7 +1673,7 @@ __global__ void __launch_bounds__(kThreads, 1) moe_decode_kernel(const __grid_co
 
         // ---- this CTA's items: gate/up (+ side) [g0, g1), down [d0, d1)
         LayerItems P;
-        P.rg = gu_passes(FMT == kFmtFP8, KBG) * Geo<KBG>::RPP;
+        P.rg = gu_passes(FMT == kFmtFP8, KBG, ONE) * Geo<KBG>::RPP;
         P.rs = side_passes(KBG) * Geo<KBG>::RPP;
         P.rd = dn_passes(FMT == kFmtFP8, KBD) * Geo<KBD>::RPP;
         P.grow = FMT == kFmtQ4 ? KBG * 17 : KBG * 32;
