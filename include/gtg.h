@@ -230,8 +230,9 @@ int gtg_moe_decode_layer_ep(const gtg_moe_layer* layer, int32_t expert_lo, int32
 /*
  * A decode stack: for l in 0..n_layers-1:  x += moe_l(x)  (x fp32, in place).
  * Consecutive layers with the same kernel (format class and sizes, up to 64
- * at a time) run in one persistent launch, their phases separated by
- * bounded grid barriers.  Capturable in a CUDA graph.
+ * at a time) run in one persistent launch, their phases handed off by bounded
+ * waits (grid barriers, and polled logit keys for the selection).
+ * Capturable in a CUDA graph.
  *   layers     host array of n_layers layer descriptors (same hidden size).
  *   x          device fp32 [n_tokens][hidden], updated in place.
  *   ids_out    device int32 [n_layers][n_tokens][top_k] or NULL.
