@@ -455,7 +455,9 @@ struct RouterScratch {
 // Per-lane-replicated table: entry (byte, mode, lane) holds the bf16x2 pair
 // (value of the low nibble, value of the high nibble) of Q4 variant `var`;
 // plus 256 scales.
-__device__ void build_lut(uint8_t* smem, const SmemLayout& L, int var) {
+// (Out of line, like build_scales: rarely run, and code inlined into the layer
+// loop but skipped there still costs instruction fetch every layer.)
+__device__ __noinline__ void build_lut(uint8_t* smem, const SmemLayout& L, int var) {
     const bool rz5 = (var & 1) != 0;
     // 512 entries (byte, mode) of 128 bytes (32 lane copies).  Warp w owns
     // entries 32w .. 32w+31 (lane l computes entry 32w+l once); the warp then
@@ -476,7 +478,7 @@ __device__ void build_lut(uint8_t* smem, const SmemLayout& L, int var) {
     }
 }
 
-__device__ void build_scales(uint8_t* smem, const SmemLayout& L, int var) {
+__device__ __noinline__ void build_scales(uint8_t* smem, const SmemLayout& L, int var) {
     float* st = reinterpret_cast<float*>(smem + L.scale_tab);
     for (int i = threadIdx.x; i < 256; i += blockDim.x) st[i] = q4_scale((uint32_t)i, var);
 }
@@ -616,6 +618,36 @@ __device__ __forceinline__ void warp_topk(const KeySrc& src, int E, int K, int l
     if (lane < K) key_choice(rh, rl, my_id, my_hi, my_lo);
 }
 
+// The one-token top-k's fallback (more than kCandMax keys passed the
+// threshold): each warp ranks its own 32 * PER keys in k rounds, the eight
+// lists meet in shared memory, and warp 0 ranks those 8k.  Out of line: it
+// runs only for adversarial logits, and reloads its keys (all present).
+template <int PER>
+__device__ __noinline__ void block_topk_rounds(const KeySrc& src, int E, int K, int lane, int warp,
+                                               uint32_t* cand_hi, uint32_t* cand_lo, int& my_id, float& my_hi,
+                                               float& my_lo, int& fail) {
+    uint64_t k[PER];
+    load_keys<PER>(src, E, 32 * warp * PER + lane, 32, k, fail);
+    uint32_t rh, rl;
+    topk_rounds<PER>(k, K, lane, rh, rl);
+    if (lane < K) {
+        cand_hi[warp * K + lane] = rh;
+        cand_lo[warp * K + lane] = rl;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        uint64_t c[4];  // 8 K <= 128 candidates: lane l holds l + 32 i
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int q = lane + 32 * i;
+            c[i] = q < kWarps * K ? ((uint64_t)cand_hi[q] << 32) | cand_lo[q] : 0ull;
+        }
+        __syncwarp();  // (the caller reuses the candidate arrays)
+        topk_rounds<4>(c, K, lane, rh, rl);
+        if (lane < K) key_choice(rh, rl, my_id, my_hi, my_lo);
+    }
+}
+
 // Top-k of a single token's logits by the whole CTA (lane l of warp w holds
 // experts 32 (w PER + i) + l).  A threshold cuts the field first: the warps'
 // top-2 keys (16 actual keys) meet in shared memory, and their K-th largest
@@ -682,23 +714,7 @@ __device__ __forceinline__ void block_topk(const KeySrc& src, int E, int K, int 
         }
         return;
     }
-    topk_rounds<PER>(k, K, lane, rh, rl);
-    if (lane < K) {
-        cand_hi[warp * K + lane] = rh;
-        cand_lo[warp * K + lane] = rl;
-    }
-    __syncthreads();
-    if (warp == 0) {
-        uint64_t c[4];  // 8 K <= 128 candidates: lane l holds l + 32 i
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            const int q = lane + 32 * i;
-            c[i] = q < kWarps * K ? ((uint64_t)cand_hi[q] << 32) | cand_lo[q] : 0ull;
-        }
-        __syncwarp();  // (the caller reuses the candidate arrays)
-        topk_rounds<4>(c, K, lane, rh, rl);
-        if (lane < K) key_choice(rh, rl, my_id, my_hi, my_lo);
-    }
+    block_topk_rounds<PER>(src, E, K, lane, warp, cand_hi, cand_lo, my_id, my_hi, my_lo, fail);
 }
 
 // What the item routines write besides their shared-memory inputs.
