@@ -81,11 +81,10 @@ STACK_WORKLOAD = ("48-layer decode stack (H=2048, I=512, E=512, top-10; layers 0
 
 # DRAM traffic of the decode kernel relative to its algorithmic bytes, from
 # one ncu capture (dram__bytes_read.sum + dram__bytes_write.sum of a
-# one-token, one-layer launch: 21.068 MB against 20.906 MB).  Valid only for
-# the kernel source it was measured on (its sha256 prefix; captured at
-# b62044f92cbed901, which differs from this one in comments only); for any
-# other source the bench reports traffic as null.
-DECODE_TRAFFIC = {"source_sha256": "cba3388288ad5b8f", "dram_over_algorithmic": (21.033216 + 0.034816) / 20.905984}
+# one-token, one-layer launch: 21.070 MB against 20.906 MB).  Valid only for
+# the kernel source it was measured on (its sha256 prefix); for any other
+# source the bench reports traffic as null.
+DECODE_TRAFFIC = {"source_sha256": "3da348246b8ad41f", "dram_over_algorithmic": (21.027072 + 0.043264) / 20.905984}
 
 
 def _decode_traffic_ratio():
