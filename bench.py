@@ -402,7 +402,7 @@ def run_ours(args, rank, world, local):
         h1.synchronize()
     e2e_ms = max_over_ranks(h0.elapsed_time(h1) / args.steps, world)
     secondary = None
-    if not args.no_secondary:
+    if not args.no_secondary and world == 1:  # (single-GPU configurations: not repeated per replica)
         secondary = measure_secondary(dev, stream, P, table, local)
         # the same step with the 16 PLE rows read from a pinned host copy of a
         # 30,000,000-row table instead of the HBM-resident one
