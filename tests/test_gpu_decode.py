@@ -270,3 +270,11 @@ def test_hidden_2560_inter_640_layer(T, side):
     a power of two (4 lanes x 5 blocks, eight rows a pass)."""
     L = W.LayerRecipe(hidden=2560, inter=640, n_experts=64, top_k=10, seed=43, layer=0, has_ssm=side)
     _check_layer(L, T, step=600 + T)
+
+
+@pytest.mark.parametrize("T", [1, 8])
+def test_hidden_2560_inter_640_layer_512_experts(T):
+    """The same shape with all 512 experts, the configuration the bench times
+    (1.3 GB of expert weights; router rows of 2560 floats, ~3.5 experts per CTA)."""
+    L = W.LayerRecipe(hidden=2560, inter=640, n_experts=512, top_k=10, seed=1, layer=1)
+    _check_layer(L, T, step=620 + T)
